@@ -1,0 +1,336 @@
+/*
+ * fqr_oracle.c -- plain, slow, obviously correct CPU oracle of the fused
+ * pre-attention preparation path.  TEST INFRASTRUCTURE ONLY (see the header):
+ * nothing in the product path includes, links or calls this file.
+ *
+ * Build: gcc -std=c11 -O2 -ffp-contract=off -fno-fast-math (no FMA
+ * contraction: every product and every sum is rounded to fp32 on its own).
+ *
+ * Sources (pages about the method, cited by title and section):
+ *  [FI]  FlashInfer PR #5956, "fused QK RMSNorm + NeoX RoPE + FP8 E4M3
+ *        quantize + NHD paged-KV append", sections "Contract", "What changes"
+ *        (test list) and the review thread on device-side validation.
+ *  [TRT] TensorRT-LLM PR #16024 "Fuse Qwen3.5 gated QKV preprocessing",
+ *        review excerpt of the fused QK norm (rsqrt(sum_sq / head_size + eps)).
+ *  [SGL] SGLang PR #43425 (fused Q/K RMSNorm + RoPE on SM100), "Modifications".
+ *  [VLLM] vLLM issue #24678 "ROPE + KV-Cache-Write + pre-attn prepare-ops
+ *        fusion" (MLA latent concat, interleaved RoPE for DeepSeek R1).
+ *
+ * parity pinned: every function below is checked by tests/test_oracle_*.py
+ * against closed forms, invariants, exhaustive brute force (encoders) or an
+ * inverse-direction brute-force model (slots, tails, flags).
+ */
+#include "fqr_oracle.h"
+
+#include <math.h>
+#include <string.h>
+
+#define D FQRO_HEAD_DIM
+
+/* ------------------------------------------------------------------------ */
+/* Formats                                                                   */
+/* ------------------------------------------------------------------------ */
+
+/* BF16 is the top half of an IEEE binary32: widening is exact. */
+float fqro_bf16_to_f32(uint16_t bits) {
+  uint32_t u = (uint32_t)bits << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* Round-to-nearest, ties-to-even, from binary32 to bfloat16 (8-bit
+ * significand, same exponent range).  Computed from the definition: find the
+ * binade of |x|, count quanta of that binade in exact double arithmetic, round
+ * the count to the nearest integer (ties to even), and rebuild.  Overflow past
+ * the largest finite value goes to infinity, NaN stays a (quiet) NaN. */
+uint16_t fqro_f32_to_bf16_rne(float x) {
+  uint32_t u;
+  memcpy(&u, &x, 4);
+  if (isnan(x)) return (uint16_t)((u >> 16) | 0x0040u);
+  uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  if (isinf(x)) return (uint16_t)(sign | 0x7F80u);
+  double a = fabs((double)x);
+  if (a == 0.0) return sign;
+  int e;
+  (void)frexp(a, &e);
+  int E = e - 1;                       /* a in [2^E, 2^(E+1)) */
+  if (E < -126) E = -126;              /* subnormal binade spacing */
+  double quantum = ldexp(1.0, E - 7);  /* 7 stored fraction bits */
+  double r = rint(a / quantum) * quantum;
+  if (r >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7F80u);
+  float rf = (float)r;                 /* exact: r has <= 8 significant bits */
+  uint32_t ur;
+  memcpy(&ur, &rf, 4);
+  return (uint16_t)(sign | (uint16_t)(ur >> 16));
+}
+
+/* OCP FP8 E4M3 ("fn" variant): 1 sign, 4 exponent (bias 7), 3 fraction bits;
+ * no infinities; S.1111.111 is NaN; largest finite 448 = S.1111.110;
+ * subnormals m * 2^-9.  Round to nearest, ties to even on the fraction, and
+ * saturate: every |x| >= 448 (infinity included) becomes +-448, as the
+ * satfinite conversion the FlashInfer page names ("RN satfinite FP8") does.
+ * NaN becomes 0x7F. */
+uint8_t fqro_f32_to_e4m3_rn_satfinite(float x) {
+  if (isnan(x)) return 0x7F;
+  uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  double a = fabs((double)x);
+  if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+  if (a == 0.0) return sign;
+  int e;
+  (void)frexp(a, &e);
+  int E = e - 1;
+  if (E < -6) E = -6;                  /* below 2^-6 the spacing is 2^-9 */
+  double quantum = ldexp(1.0, E - 3);  /* 3 fraction bits */
+  double n = rint(a / quantum);        /* exact division by a power of two */
+  if (E == -6 && n < 8.0) return (uint8_t)(sign | (uint8_t)n); /* subnormal */
+  if (n >= 16.0) {                     /* rounded up into the next binade */
+    E += 1;
+    n = 8.0;
+  }
+  return (uint8_t)(sign | (uint8_t)(((E + 7) << 3) | ((int)n - 8)));
+}
+
+void fqro_f32_to_e4m3_array(const float* x, uint8_t* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = fqro_f32_to_e4m3_rn_satfinite(x[i]);
+}
+
+void fqro_f32_to_bf16_array(const float* x, uint16_t* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = fqro_f32_to_bf16_rne(x[i]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Per-head steps                                                            */
+/* ------------------------------------------------------------------------ */
+
+/* RMSNorm over one head ([TRT] review excerpt; [FI] "per-head RMSNorm eps
+ * 1e-6"): mean square over all n elements, eps inside the square root, then
+ * scale and weight.  Sequential fp32 sum of rounded squares. */
+void fqro_rmsnorm(const float* x, const float* w, int n, float eps, float* y) {
+  float ss = 0.0f;
+  for (int i = 0; i < n; ++i) {
+    float sq = x[i] * x[i];
+    ss = ss + sq;
+  }
+  float ms = ss / (float)n;
+  float inv = 1.0f / sqrtf(ms + eps);
+  for (int i = 0; i < n; ++i) {
+    float t = x[i] * inv;
+    y[i] = w ? t * w[i] : t;
+  }
+}
+
+/* NeoX ("rotate half") RoPE ([SGL] "full-width NeoX rotation", [FI] "NeoX
+ * RoPE"): element i pairs with i + rot/2; the cache row is [cos | sin]. */
+void fqro_rope_neox(float* y, const float* cs_row, int rot) {
+  int half = rot / 2;
+  for (int i = 0; i < half; ++i) {
+    float c = cs_row[i], s = cs_row[half + i];
+    float a = y[i], b = y[i + half];
+    float ac = a * c, bs = b * s, bc = b * c, as = a * s;
+    y[i] = ac - bs;
+    y[i + half] = bc + as;
+  }
+}
+
+/* GPT-J (interleaved) RoPE ([VLLM] "RoPE/NoPE interleaved" for DeepSeek R1):
+ * element 2i pairs with 2i + 1; the cache row is [cos | sin]. */
+void fqro_rope_gptj(float* y, const float* cs_row, int rot) {
+  int half = rot / 2;
+  for (int i = 0; i < half; ++i) {
+    float c = cs_row[i], s = cs_row[half + i];
+    float a = y[2 * i], b = y[2 * i + 1];
+    float ac = a * c, bs = b * s, bc = b * c, as = a * s;
+    y[2 * i] = ac - bs;
+    y[2 * i + 1] = bc + as;
+  }
+}
+
+static void rope(float* y, const float* cs_row, int rot, int style) {
+  if (style == 0)
+    fqro_rope_neox(y, cs_row, rot);
+  else
+    fqro_rope_gptj(y, cs_row, rot);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Validation ([FI] "Contract": malformed q_indptr -> all flags -1 and nothing */
+/* written; the review thread adds seq_lens < new tokens, page-table overrun  */
+/* and cos/sin row overrun to the same rule).                                */
+/* ------------------------------------------------------------------------ */
+int fqro_validate(const int32_t* q_indptr, const int32_t* seq_lens, int32_t B,
+                  int32_t T, int32_t max_pages, int32_t page_size,
+                  int32_t cos_sin_rows, const int64_t* positions) {
+  if (q_indptr[0] != 0) return 1;
+  if (q_indptr[B] != T) return 1;
+  for (int32_t b = 0; b < B; ++b) {
+    int64_t lo = q_indptr[b], hi = q_indptr[b + 1], L = seq_lens[b];
+    if (hi < lo) return 1;
+    if (L < hi - lo) return 1;  /* derived positions would go negative */
+    if (L > (int64_t)max_pages * page_size) return 1;
+    if (!positions && L > cos_sin_rows) return 1;
+  }
+  if (positions) {
+    for (int32_t t = 0; t < T; ++t)
+      if (positions[t] < 0 || positions[t] >= cos_sin_rows) return 1;
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Paged append ([FI] "Contract")                                            */
+/* ------------------------------------------------------------------------ */
+
+static void widen_head(const uint16_t* src, float* x, int n) {
+  for (int i = 0; i < n; ++i) x[i] = fqro_bf16_to_f32(src[i]);
+}
+
+int fqro_append_paged(const fqro_append_args* a) {
+  if (fqro_validate(a->q_indptr, a->seq_lens, a->B, a->T, a->max_pages,
+                    a->page_size, a->cos_sin_rows, a->positions)) {
+    for (int32_t b = 0; b < a->B; ++b) a->flags[b] = -1;
+    return 1;
+  }
+  const int P = a->page_size;
+  const int fp8 = a->quant_policy != 0;
+  float wq[D], wk[D], x[D], y[D];
+  if (a->q_norm_w) widen_head(a->q_norm_w, wq, D);
+  if (a->k_norm_w) widen_head(a->k_norm_w, wk, D);
+
+  for (int32_t b = 0; b < a->B; ++b) {
+    int64_t lo = a->q_indptr[b], hi = a->q_indptr[b + 1], L = a->seq_lens[b];
+    for (int64_t r = lo; r < hi; ++r) {
+      /* seq_lens is the length after the append: token r sits at
+       * r + L - q_indptr[b + 1]; the KV slot always uses that position. */
+      int64_t p_slot = r + L - hi;
+      int64_t pos = a->positions ? a->positions[r] : p_slot;
+      int64_t page = a->page_table[(int64_t)b * a->max_pages + p_slot / P];
+      int64_t row = p_slot % P;
+      const float* cs = a->cos_sin + pos * a->rot_dim;
+      const uint16_t* src = a->qkv + r * a->row_stride;
+
+      for (int h = 0; h < a->Hq; ++h) {
+        widen_head(src + (int64_t)h * D, x, D);
+        if (a->q_norm_w)
+          fqro_rmsnorm(x, wq, D, a->eps, y);
+        else
+          memcpy(y, x, sizeof y);
+        rope(y, cs, a->rot_dim, a->rope_style);
+        int64_t o = (r * a->Hq + h) * D;
+        if (a->quant_policy == 0) {
+          uint16_t* q = (uint16_t*)a->out_q + o;
+          for (int i = 0; i < D; ++i) q[i] = fqro_f32_to_bf16_rne(y[i]);
+        } else if (a->quant_policy == 1) {
+          /* dynamic per-token/per-head scale: max(max|q|, 1e-6) / upper_max,
+           * payload q / q_scale ([FI] "Contract" and test list) */
+          float amax = 0.0f;
+          for (int i = 0; i < D; ++i) amax = fmaxf(amax, fabsf(y[i]));
+          float qs = fmaxf(amax, 1e-6f) / a->upper_max;
+          a->q_scale[r * a->Hq + h] = qs;
+          uint8_t* q = (uint8_t*)a->out_q + o;
+          for (int i = 0; i < D; ++i) q[i] = fqro_f32_to_e4m3_rn_satfinite(y[i] / qs);
+        } else {
+          /* static per-tensor: payload q * q_scale_inv */
+          uint8_t* q = (uint8_t*)a->out_q + o;
+          for (int i = 0; i < D; ++i)
+            q[i] = fqro_f32_to_e4m3_rn_satfinite(y[i] * a->q_scale_inv);
+        }
+      }
+      for (int kh = 0; kh < a->Hkv; ++kh) {
+        int64_t ko = page * a->k_page_stride + (row * a->Hkv + kh) * D;
+        int64_t vo = page * a->v_page_stride + (row * a->Hkv + kh) * D;
+        /* K head */
+        widen_head(src + (int64_t)(a->Hq + kh) * D, x, D);
+        if (a->k_norm_w)
+          fqro_rmsnorm(x, wk, D, a->eps, y);
+        else
+          memcpy(y, x, sizeof y);
+        rope(y, cs, a->rot_dim, a->rope_style);
+        if (!fp8) {
+          uint16_t* k = (uint16_t*)a->k_cache + ko;
+          for (int i = 0; i < D; ++i) k[i] = fqro_f32_to_bf16_rne(y[i]);
+        } else {
+          uint8_t* k = (uint8_t*)a->k_cache + ko;
+          for (int i = 0; i < D; ++i) k[i] = fqro_f32_to_e4m3_rn_satfinite(y[i] / a->k_scale);
+        }
+        /* V head: a bit copy in BF16, x / v_scale in FP8 */
+        const uint16_t* vs = src + (int64_t)(a->Hq + a->Hkv + kh) * D;
+        if (!fp8) {
+          memcpy((uint16_t*)a->v_cache + vo, vs, D * sizeof(uint16_t));
+        } else {
+          uint8_t* v = (uint8_t*)a->v_cache + vo;
+          for (int i = 0; i < D; ++i)
+            v[i] = fqro_f32_to_e4m3_rn_satfinite(fqro_bf16_to_f32(vs[i]) / a->v_scale);
+        }
+      }
+    }
+  }
+
+  /* Rows [last + 1, page_size) of every request's last page are zeroed in
+   * both caches ([FI] "Contract"); a request with L == 0 has no last page. */
+  const int64_t esize = fp8 ? 1 : 2;
+  for (int32_t b = 0; b < a->B; ++b) {
+    int64_t L = a->seq_lens[b];
+    if (L <= 0) continue;
+    int64_t last = (L - 1) % P;
+    int64_t page = a->page_table[(int64_t)b * a->max_pages + (L - 1) / P];
+    for (int64_t row = last + 1; row < P; ++row) {
+      int64_t ko = page * a->k_page_stride + row * a->Hkv * D;
+      int64_t vo = page * a->v_page_stride + row * a->Hkv * D;
+      memset((char*)a->k_cache + ko * esize, 0, (size_t)(a->Hkv * D * esize));
+      memset((char*)a->v_cache + vo * esize, 0, (size_t)(a->Hkv * D * esize));
+    }
+  }
+  for (int32_t b = 0; b < a->B; ++b) a->flags[b] = 0;
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* MLA latent concat ([VLLM] concat_and_cache_mla; interleaved RoPE on the    */
+/* rope part of Q and on k_pe; latent row = [kv_c | rope(k_pe)])             */
+/* ------------------------------------------------------------------------ */
+int fqro_concat_mla_cache(const fqro_mla_args* a) {
+  if (fqro_validate(a->q_indptr, a->seq_lens, a->B, a->T, a->max_blocks,
+                    a->block_size, a->cos_sin_rows, a->positions)) {
+    for (int32_t b = 0; b < a->B; ++b) a->flags[b] = -1;
+    return 1;
+  }
+  const int R = a->rope_dim, K = a->kv_lora_rank, W = K + R;
+  float y[512];
+  if (R > 512) return 2;
+  for (int32_t b = 0; b < a->B; ++b) {
+    int64_t lo = a->q_indptr[b], hi = a->q_indptr[b + 1], L = a->seq_lens[b];
+    for (int64_t r = lo; r < hi; ++r) {
+      int64_t p_slot = r + L - hi;
+      int64_t pos = a->positions ? a->positions[r] : p_slot;
+      int64_t blk = a->block_table[(int64_t)b * a->max_blocks + p_slot / a->block_size];
+      int64_t row = p_slot % a->block_size;
+      const float* cs = a->cos_sin + pos * R;
+      /* Q: rotate the rope part in place, the nope part is left as it is */
+      for (int h = 0; h < a->Hq; ++h) {
+        uint16_t* qp = a->q + r * a->q_token_stride + h * a->q_head_stride + a->nope_dim;
+        widen_head(qp, y, R);
+        rope(y, cs, R, a->rope_style);
+        for (int i = 0; i < R; ++i) qp[i] = fqro_f32_to_bf16_rne(y[i]);
+      }
+      /* latent row */
+      int64_t base = (blk * a->block_size + row) * W;
+      const uint16_t* kc = a->kv_c + r * a->kv_c_stride;
+      widen_head(a->k_pe + r * a->k_pe_stride, y, R);
+      rope(y, cs, R, a->rope_style);
+      if (a->cache_fp8) {
+        uint8_t* dst = (uint8_t*)a->latent_cache + base;
+        for (int i = 0; i < K; ++i)
+          dst[i] = fqro_f32_to_e4m3_rn_satfinite(fqro_bf16_to_f32(kc[i]) / a->kv_scale);
+        for (int i = 0; i < R; ++i)
+          dst[K + i] = fqro_f32_to_e4m3_rn_satfinite(y[i] / a->kv_scale);
+      } else {
+        uint16_t* dst = (uint16_t*)a->latent_cache + base;
+        memcpy(dst, kc, (size_t)K * sizeof(uint16_t));
+        for (int i = 0; i < R; ++i) dst[K + i] = fqro_f32_to_bf16_rne(y[i]);
+      }
+    }
+  }
+  for (int32_t b = 0; b < a->B; ++b) a->flags[b] = 0;
+  return 0;
+}
