@@ -1,0 +1,603 @@
+#!/usr/bin/env python
+"""Benchmark of the fused QK-norm + RoPE + quant + paged-append path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one fused call (one kernel: validation, Q/K RMSNorm, RoPE,
+quantisation, paged K/V scatter, last-page tail zeroing, flags) over one batch
+of the Qwen3-style decode workload: 128 requests x 1 new token, Hq 32 / Hkv 8,
+head_dim 128, page 16, 1M-slot BF16 NHD cache.  Inputs are synthetic and
+seeded (workloads.py).  Each step uses its own replica of the step inputs
+(packed QKV, metadata, page table, out_q) and writes pages of its own, with
+enough replicas that the per-step data rotated over in the timed region is
+larger than L2 (126 MB); the timed launches are replayed from CUDA graphs.
+
+Rank 0 prints one JSON line.  `value` = tokens/s over all ranks (the
+max-over-ranks device time of K steps); `roofline` = algorithmic bytes per
+launch / average launch time, against the measured HBM copy bandwidth;
+`e2e` = the same metric through the public API with pinned host buffers
+(host->device copies of the step's inputs and device->host copies of out_q
+and flags inside the timed region); `cpu_baseline` = the CPU oracle on a
+bounded sample; `per_config` adds the other named workloads (kernel time,
+GB/s, fraction of peak) measured the same way, outside the timed region.
+
+--impl reference times the CPU oracle (the reference arm of this build) on
+the host cores on the same workload, metric and unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "fused QKnorm+RoPE+quant+paged-append tokens/s and HBM GB/s (% of peak), 1 B200"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+MAIN_WORKLOAD = "qwen3_decode_bf16"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200000)
+    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=MAIN_WORKLOAD, choices=sorted(workloads.APPEND_CONFIGS))
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU budget of the oracle baseline sample")
+    ap.add_argument("--e2e-steps", type=int, default=3000)
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: copy, read+write)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "qk_norm_rope_token_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    if it was captured on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"append_paged_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("bench-key:"):
+                k, _, v = line[len("bench-key:"):].strip().partition("=")
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_sources") != kernel_source_hash():
+        return None
+    try:
+        return int(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of one GPU during the timed region."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fd, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        self.t0 = self.t1 = None
+
+    def mark(self, start: bool):
+        if start:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        os.close(self.fd)
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                    rows.append((ts, float(parts[1]), float(parts[2]), parts[3], parts[5:9]))
+                except (ValueError, IndexError):
+                    continue
+        os.unlink(self.path)
+        inside = [r for r in rows if self.t0 and self.t1 and self.t0 - 0.15 <= r[0] <= self.t1 + 0.15]
+        window = "timed region"
+        if len(inside) < 3:
+            inside, window = rows, "warm-up and timed region"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in inside for n, v in zip(names, r[4]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside), "window": window}
+
+
+def gpu_smi_id(torch, dev) -> str:
+    """nvidia-smi --id of the GPU torch calls `dev` (its UUID)."""
+    props = torch.cuda.get_device_properties(dev)
+    u = str(getattr(props, "uuid", ""))
+    if u and not u.startswith("GPU-"):
+        u = "GPU-" + u
+    return u or str(dev.index)
+
+
+# -------------------------------------------------------- device workloads
+
+class AppendBench:
+    """R replicas of one append workload sharing one pair of KV caches."""
+
+    def __init__(self, name, torch, fqr, device, min_bytes=3 * L2_BYTES, max_replicas=64,
+                 seed_offset=0):
+        self.torch, self.fqr, self.dev = torch, fqr, device
+        base = workloads.APPEND_CONFIGS[name]()
+        self.name = base.name
+        per = workloads.append_bytes(base)["total"]
+        self.R = int(min(max_replicas, max(2, math.ceil(min_bytes / per))))
+        ws = []
+        for r in range(self.R):
+            sd = base.seed + seed_offset + 7919 * r
+            ws.append(base if sd == base.seed else workloads.APPEND_CONFIGS[name](seed=sd))
+        self.ws = ws
+        self.bytes = [workloads.append_bytes(w)["total"] for w in ws]
+        self.T = base.T
+        w0 = ws[0]
+        es = w0.kv_esize
+        dt = torch.int16 if es == 2 else torch.uint8
+        shape = (w0.num_pages, w0.page_size, w0.Hkv, 128)
+        self.k_cache = torch.empty(shape, dtype=dt, device=device)
+        self.v_cache = torch.empty(shape, dtype=dt, device=device)
+        self.cs = self._d(w0.cos_sin)
+        self.qw = self._d(w0.q_norm_w)
+        self.kw = self._d(w0.k_norm_w)
+        self.scales = {k: torch.tensor([v], dtype=torch.float32, device=device)
+                       for k, v in (("q_scale_inv", w0.q_scale_inv), ("k_scale", w0.k_scale),
+                                    ("v_scale", w0.v_scale))}
+        self.reps = []
+        for w in ws:
+            st = dict(qkv=self._d(w.qkv), q_indptr=self._d(w.q_indptr),
+                      seq_lens=self._d(w.seq_lens), page_table=self._d(w.page_table),
+                      out_q=torch.empty((w.T, w.Hq, 128), dtype=dt if w.quant_policy == 0
+                                        else torch.uint8, device=device),
+                      q_scale=torch.empty((max(w.T, 1), w.Hq), dtype=torch.float32,
+                                          device=device),
+                      flags=torch.empty((w.B,), dtype=torch.int32, device=device))
+            st["params"] = self._params(w, st)
+            self.reps.append(st)
+
+    def _d(self, a):
+        if a is None:
+            return None
+        t = self.torch.from_numpy(np.ascontiguousarray(a))
+        if t.dtype == self.torch.uint16:
+            t = t.view(self.torch.int16)
+        return t.to(self.dev)
+
+    def kw_for(self, w, st):
+        return dict(q_norm_w=self.qw, k_norm_w=self.kw, eps=w.eps, rope_style=w.rope_style,
+                    rot_dim=w.rot_dim, quant_policy=w.quant_policy,
+                    q_scale=st["q_scale"] if w.quant_policy == 1 else None,
+                    q_scale_inv=self.scales["q_scale_inv"] if w.quant_policy == 2 else None,
+                    k_scale=self.scales["k_scale"] if w.quant_policy else None,
+                    v_scale=self.scales["v_scale"] if w.quant_policy else None,
+                    upper_max=w.upper_max)
+
+    def _params(self, w, st):
+        return self.fqr.append_params(st["qkv"], self.cs, st["q_indptr"], st["seq_lens"],
+                                      st["page_table"], self.k_cache, self.v_cache, st["out_q"],
+                                      st["flags"], **self.kw_for(w, st))
+
+    def launch(self, i, stream_handle):
+        rc = self.fqr.append_paged_raw(self.reps[i % self.R]["params"], stream_handle)
+        if rc != 0:
+            raise self.fqr.FqrError(rc)
+
+    def check_flags(self):
+        for st in self.reps:
+            assert int(st["flags"].abs().max()) == 0, "a replica was flagged"
+
+
+class MlaBench:
+    def __init__(self, torch, fqr, device, min_bytes=3 * L2_BYTES, max_replicas=256):
+        self.torch, self.fqr, self.dev = torch, fqr, device
+        base = workloads.mla_decode()
+        self.name = base.name
+        per = workloads.mla_bytes(base)["total"]
+        self.R = int(min(max_replicas, max(2, math.ceil(min_bytes / per))))
+        self.ws = [base] + [workloads.make_mla(seed=base.seed + 7919 * r, n_new=[1] * base.B,
+                                               seq_lens=base.seq_lens, Hq=base.Hq,
+                                               block_size=base.block_size,
+                                               max_blocks=base.max_blocks,
+                                               cos_sin_rows=base.cos_sin_rows)
+                            for r in range(1, self.R)]
+        self.bytes = [workloads.mla_bytes(w)["total"] for w in self.ws]
+        self.T = base.T
+        self.latent = torch.empty((base.num_blocks, base.block_size, base.width),
+                                  dtype=torch.uint8, device=device)
+        self.cs = self._d(base.cos_sin)
+        self.scale = torch.tensor([base.kv_scale], dtype=torch.float32, device=device)
+        self.params = []
+        self.keep = []
+        for w in self.ws:
+            q, kv_c, k_pe = self._d(w.q), self._d(w.kv_c), self._d(w.k_pe)
+            ind, sl, bt = self._d(w.q_indptr), self._d(w.seq_lens), self._d(w.block_table)
+            flags = torch.empty((w.B,), dtype=torch.int32, device=device)
+            self.keep.append((q, kv_c, k_pe, ind, sl, bt, flags))
+            self.params.append(fqr.mla_params(q, kv_c, k_pe, self.cs, ind, sl, bt, self.latent,
+                                              flags, nope_dim=w.nope_dim,
+                                              rope_style=w.rope_style, kv_scale=self.scale))
+
+    _d = AppendBench._d
+
+    def launch(self, i, stream_handle):
+        rc = self.fqr.concat_mla_cache_raw(self.params[i % self.R], stream_handle)
+        if rc != 0:
+            raise self.fqr.FqrError(rc)
+
+
+def time_launches(torch, bench, steps, warmup, graph_chunk=1000, barrier=None, marks=None):
+    """Warm up, then time exactly `steps` launches (replayed from CUDA graphs
+    of up to `graph_chunk` launches, cycling over the replicas) with CUDA
+    events on the launching stream.  Returns (elapsed_ms, bytes)."""
+    stream = torch.cuda.current_stream()
+    h = stream.cuda_stream
+    for i in range(warmup):
+        bench.launch(i, h)
+    torch.cuda.synchronize()
+
+    def capture(n, first):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            hs = torch.cuda.current_stream().cuda_stream
+            for i in range(n):
+                bench.launch(first + i, hs)
+        return g
+
+    chunk = max(1, min(graph_chunk, steps))
+    # a chunk that is a multiple of R keeps every replay's replica set identical
+    if chunk >= bench.R:
+        chunk -= chunk % bench.R
+    full, rest = divmod(steps, chunk)
+    g_full = capture(chunk, 0) if full else None
+    g_rest = capture(rest, 0) if rest else None
+    # replay once untimed (graph upload)
+    if g_full is not None:
+        g_full.replay()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if barrier is not None:
+        barrier()
+    torch.cuda.synchronize()
+    if marks is not None:
+        marks(True)
+    start.record(stream)
+    for _ in range(full):
+        g_full.replay()
+    if g_rest is not None:
+        g_rest.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if marks is not None:
+        marks(False)
+    if barrier is not None:
+        barrier()
+    ms = start.elapsed_time(end)
+    nbytes = sum(bench.bytes[i % bench.R] for i in range(chunk)) * full + \
+        sum(bench.bytes[i % bench.R] for i in range(rest))
+    del g_full, g_rest
+    return ms, nbytes
+
+
+def e2e_measure(torch, fqr, bench, steps):
+    """Same metric through the public API with pinned host buffers."""
+    w0 = bench.ws[0]
+    dev = bench.dev
+    R = min(bench.R, 8)
+    host_in, host_out = [], []
+    for w in bench.ws[:R]:
+        hi = {"qkv": torch.from_numpy(w.qkv.view(np.int16)).pin_memory(),
+              "q_indptr": torch.from_numpy(w.q_indptr).pin_memory(),
+              "seq_lens": torch.from_numpy(w.seq_lens).pin_memory(),
+              "page_table": torch.from_numpy(w.page_table).pin_memory()}
+        host_in.append(hi)
+        ho = {"out_q": torch.empty(bench.reps[0]["out_q"].shape,
+                                   dtype=bench.reps[0]["out_q"].dtype).pin_memory(),
+              "flags": torch.empty((w.B,), dtype=torch.int32).pin_memory()}
+        if w.quant_policy == 1:
+            ho["q_scale"] = torch.empty((w.T, w.Hq), dtype=torch.float32).pin_memory()
+        host_out.append(ho)
+    dev_in = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in host_in[0].items()}
+    dev_out = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in host_out[0].items()}
+    kw = bench.kw_for(w0, {"q_scale": dev_out.get("q_scale")})
+    kw.pop("q_scale", None)
+    h2d = sum(v.numel() * v.element_size() for v in host_in[0].values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out[0].values())
+
+    def step(i):
+        fqr.append_paged_from_host(host_in[i % R], dev_in, host_out[i % R], dev_out,
+                                   cos_sin_cache=bench.cs, k_cache=bench.k_cache,
+                                   v_cache=bench.v_cache, **kw)
+
+    for i in range(20):
+        step(i)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    assert int(host_out[(steps - 1) % R]["flags"].abs().max()) == 0
+    return {"value": bench.T * steps / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+# ----------------------------------------------------------- CPU baselines
+
+def oracle_sample(w, budget_s, max_calls=None):
+    """Time the oracle as it stands on whole calls of workload w (host caches
+    allocated lazily: only the pages a call touches are materialised)."""
+    import oracle
+    es = w.kv_esize
+    dt = np.uint16 if es == 2 else np.uint8
+    shape = (w.num_pages, w.page_size, w.Hkv, 128)
+    kc = np.zeros(shape, dt)
+    vc = np.zeros(shape, dt)
+    oq, qs, fl = oracle.new_outputs(w)
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        rc = oracle.append_paged(w, kc, vc, oq, qs if w.quant_policy == 1 else None, fl)
+        assert rc == 0
+        calls += 1
+        el = time.perf_counter() - t0
+        if (max_calls and calls >= max_calls) or (not max_calls and el >= budget_s):
+            break
+    return calls, el
+
+
+def cpu_baseline(w, budget_s):
+    calls, el = oracle_sample(w, budget_s)
+    return {"value": w.T * calls / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{calls} whole calls of {w.name} ({w.T} tokens each), "
+                      f"{el:.1f} s single-threaded C oracle (fp32, -O2, no FMA)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    w = workloads.APPEND_CONFIGS[args.workload]()
+    import oracle
+    # size each step's sample so the whole run stays within a few minutes
+    calls, el = oracle_sample(w, 0.0, max_calls=2)
+    t_call = el / calls
+    per_token = t_call / max(w.T, 1)
+    budget = 120.0
+    tokens = int(max(1, min(w.T, budget / max(1, args.steps + args.warmup) / per_token)))
+    subs = []
+    for b0 in range(0, w.B, tokens):
+        subs.append(_sub_batch(w, b0, min(w.B, b0 + tokens)))
+    es = w.kv_esize
+    dt = np.uint16 if es == 2 else np.uint8
+    kc = np.zeros((w.num_pages, w.page_size, w.Hkv, 128), dt)
+    vc = np.zeros_like(kc)
+    outs = [oracle.new_outputs(s) for s in subs]
+
+    def step(i):
+        s = subs[i % len(subs)]
+        oq, qs, fl = outs[i % len(subs)]
+        assert oracle.append_paged(s, kc, vc, oq, qs if s.quant_policy == 1 else None, fl) == 0
+        return s.T
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    toks = sum(step(i) for i in range(args.steps))
+    el = time.perf_counter() - t0
+    value = toks / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": config_block(w, None),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} steps of {tokens} request(s) x 1 token of "
+                                   f"{w.name}, single-threaded C oracle"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _sub_batch(w, b0, b1):
+    """Requests [b0, b1) of an append workload as a workload of their own."""
+    import copy
+    s = copy.copy(w)
+    lo, hi = int(w.q_indptr[b0]), int(w.q_indptr[b1])
+    s.B = b1 - b0
+    s.T = hi - lo
+    s.qkv = w.qkv[lo:hi]
+    s.q_indptr = (w.q_indptr[b0:b1 + 1] - lo).astype(np.int32)
+    s.seq_lens = w.seq_lens[b0:b1].copy()
+    s.page_table = w.page_table[b0:b1].copy()
+    s.positions = None if w.positions is None else w.positions[lo:hi]
+    return s
+
+
+def max_over_ranks(torch, dist, x: float, device) -> float:
+    """The maximum of a per-rank time over all ranks (x itself on one rank)."""
+    if dist is None or not dist.is_initialized():
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def config_block(w, bench):
+    c = {"workload": w.name, "tokens_per_step": w.T, "requests": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+         "head_dim": 128, "page_size": w.page_size, "quant_policy": w.quant_policy,
+         "io_dtype": "bf16 in, " + ("bf16" if w.quant_policy == 0 else "e4m3") + " out",
+         "parallelism": "replicas"}
+    if bench is not None:
+        c["replicas"] = bench.R
+        c["l2"] = (f"inputs larger than L2: each step uses its own replica of the step inputs "
+                   f"({bench.R} replicas, {sum(bench.bytes) / 1e6:.0f} MB rotated per cycle)")
+    return c
+
+
+# --------------------------------------------------------------------- main
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import qk_norm_rope_token_b200 as fqr
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    peak, peak_src = load_peaks()
+    bench = AppendBench(args.workload, torch, fqr, dev, seed_offset=1000 * rank)
+    sampler = ClockSampler(gpu_smi_id(torch, dev)) if rank == 0 else None
+    if sampler is not None:
+        time.sleep(1.0)   # let nvidia-smi start sampling before the warm-up
+    ms, nbytes = time_launches(torch, bench, args.steps, args.warmup, barrier=barrier,
+                               marks=sampler.mark if sampler else None)
+    bench.check_flags()
+    clocks = sampler.stop() if sampler else None
+    ms_max = max_over_ranks(torch, dist, ms, dev)
+    value = world * bench.T * args.steps / (ms_max / 1e3)
+    per_launch_s = ms / 1e3 / args.steps
+    achieved = nbytes / args.steps / per_launch_s / 1e9
+
+    e2e = e2e_measure(torch, fqr, bench, min(args.e2e_steps, max(args.steps, 1)))
+    e2e_ms = max_over_ranks(torch, dist, e2e["ms_per_step"], dev)
+    e2e["value"] = world * bench.T / (e2e_ms / 1e3)
+    per_config = None
+    if rank == 0 and not args.no_per_config:
+        per_config = measure_per_config(torch, fqr, dev, peak, args.workload)
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        cpu = cpu_baseline(bench.ws[0], args.cpu_seconds)
+    if dist is not None:
+        barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": config_block(bench.ws[0], bench),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                     "peak_source": peak_src,
+                     "bytes_per_launch": nbytes / args.steps,
+                     "kernel": "fqr::append_kernel", "timing": "CUDA events around graph "
+                     "replays of back-to-back launches; average launch = region / steps"},
+        "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks, "cpu_baseline": cpu,
+        "per_config": per_config,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def measure_per_config(torch, fqr, dev, peak, main_name, steps=20000, warmup=200):
+    out = {}
+    for name in sorted(workloads.APPEND_CONFIGS):
+        b = AppendBench(name, torch, fqr, dev)
+        n = max(200, min(steps, int(2e10 / max(b.bytes))))   # ~a few hundred ms each
+        ms, nbytes = time_launches(torch, b, n, warmup)
+        b.check_flags()
+        us = ms * 1e3 / n
+        gbs = nbytes / n / (us * 1e-6) / 1e9
+        out[name] = {"workload": b.name, "us_per_launch": us, "tokens_per_s": b.T / (us * 1e-6),
+                     "GB_per_s": gbs, "frac_of_peak": gbs / peak,
+                     "bytes_per_launch": nbytes / n, "replicas": b.R, "launches": n}
+        del b
+        torch.cuda.empty_cache()
+    m = MlaBench(torch, fqr, dev)
+    n = 20000
+    ms, nbytes = time_launches(torch, m, n, warmup)
+    us = ms * 1e3 / n
+    gbs = nbytes / n / (us * 1e-6) / 1e9
+    out["mla_decode"] = {"workload": m.name, "us_per_launch": us,
+                         "tokens_per_s": m.T / (us * 1e-6), "GB_per_s": gbs,
+                         "frac_of_peak": gbs / peak, "bytes_per_launch": nbytes / n,
+                         "replicas": m.R, "launches": n}
+    return out
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,71 @@
+"""Multi-rank plumbing of bench.py on CPU (gloo, world size 2): the timing
+reduction takes the maximum over ranks, and the reference arm runs on rank 0
+only (other ranks exit 0 without work)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.max_over_ranks(torch, dist, 10.0 + 5.0 * rank, torch.device("cpu"))
+        out[rank] = got
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+        assert dict(out) == {0: 15.0, 1: 15.0}
+
+
+def test_max_over_ranks_single_process():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(torch, None, 3.5, torch.device("cpu")) == 3.5
+
+
+def test_reference_arm_nonzero_rank_does_nothing(capsys):
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    args = bench.parse_args(["--impl", "reference", "--steps", "3", "--warmup", "1"])
+    assert bench.run_reference(args, rank=1, world=2) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_rank0_prints_one_line(capsys):
+    import json
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    args = bench.parse_args(["--impl", "reference", "--steps", "3", "--warmup", "1",
+                             "--workload", "tiny_decode_bf16"])
+    assert bench.run_reference(args, rank=0, world=1) == 0
+    lines = capsys.readouterr().out.strip().splitlines()
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["value"] > 0 and rec["unit"] == "tokens/s"
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"

@@ -1,0 +1,218 @@
+"""GPU parity of fqr_append_paged against the oracle, through the C ABI.
+
+Full-size named workloads (in the launch configuration bench.py times), the
+malformed-metadata run, and a sweep of small ragged cases spanning several
+tiles and ragged tails, plus edge cases: requests without tokens, every
+malformed predicate, the largest batch, padded rows and page strides,
+explicit positions, norm off, all 65536 BF16 inputs through the FP8 encoder,
+the reduction-scope guard, a non-default stream and CUDA-graph replay."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests._util import bf16_bits_to_f32, ulp_e4m3
+
+pytestmark = pytest.mark.gpu
+D = 128
+
+if torch.cuda.is_available():
+    from tests.gpu_harness import AppendRun, _np
+
+
+def run_and_check(w, **kw):
+    check_kw = {k: kw.pop(k) for k in list(kw) if k in ("exact_frac_min",)}
+    r = AppendRun(w, **kw)
+    r.launch()
+    rep = r.check(**check_kw)
+    return r, rep
+
+
+@pytest.mark.parametrize("name", sorted(workloads.APPEND_CONFIGS))
+def test_named_workload_parity(name):
+    w = workloads.APPEND_CONFIGS[name]()
+    _, rep = run_and_check(w)
+    print(name, rep)
+    assert not rep.get("flagged")
+
+
+def test_ragged_prefill_malformed_indptr_writes_nothing():
+    w = workloads.ragged_prefill_fp8()
+    r = AppendRun(w, q_indptr=workloads.malformed_indptr(w))
+    r.launch()
+    rep = r.check()
+    assert rep == {"flagged": True}
+    assert (r.flags.cpu().numpy() == -1).all()
+
+
+SWEEP = [
+    # (P, Hq, Hkv, policy, style, rot, norm, positions, row_pad)
+    (4, 8, 1, 0, 0, 128, True, False, 0),
+    (16, 32, 8, 0, 0, 128, True, False, 64),
+    (64, 64, 8, 1, 0, 128, True, False, 0),
+    (16, 64, 8, 2, 0, 128, True, False, 0),
+    (128, 8, 1, 1, 0, 128, True, True, 0),
+    (16, 4, 4, 2, 1, 128, True, False, 8),
+    (64, 16, 2, 1, 1, 64, True, False, 0),
+    (16, 6, 2, 0, 1, 2, False, False, 0),
+    (32, 12, 4, 2, 0, 128, False, True, 0),
+    (1, 8, 8, 1, 0, 128, True, False, 0),
+    (16, 128, 8, 1, 0, 128, True, False, 0),
+]
+
+
+@pytest.mark.parametrize("P,Hq,Hkv,policy,style,rot,norm,pos,pad", SWEEP)
+@pytest.mark.parametrize("seed", [1, 2])
+def test_small_ragged_sweep(P, Hq, Hkv, policy, style, rot, norm, pos, pad, seed):
+    rng = np.random.default_rng(seed * 1000 + P + Hq)
+    B = 7
+    n = rng.integers(0, 40, B)
+    n[rng.integers(0, B)] = 0
+    prior = rng.integers(0, 3 * P + 5, B)
+    L = prior + n
+    max_pages = int(np.ceil(L.max() / P)) + 1
+    rows = int(L.max()) + 7
+    positions = None
+    if pos:
+        positions = rng.integers(0, rows, int(n.sum()))
+    w = workloads.make_append(seed=seed, n_new=n, seq_lens=L, Hq=Hq, Hkv=Hkv, page_size=P,
+                              max_pages=max_pages, num_pages=B * max_pages + 3,
+                              quant_policy=policy, qkv_sigma=2.0, norm=norm, rot_dim=rot,
+                              rope_style=style, cos_sin_rows=rows, row_pad=pad,
+                              positions=positions, q_scale_inv=1 / 0.05, k_scale=0.05,
+                              v_scale=0.05)
+    _, rep = run_and_check(w, exact_frac_min=0.95)
+    if not norm:
+        # without the norm both sides evaluate identical fp32 expressions
+        assert rep["q_exact_frac"] == 1.0 and rep.get("k_exact_frac", 1.0) == 1.0
+
+
+def test_requests_without_tokens_only_tails_and_flags():
+    w = workloads.make_append(seed=3, n_new=[0, 0, 0, 0], seq_lens=[0, 5, 16, 33], Hq=8, Hkv=2,
+                              page_size=16, max_pages=3, quant_policy=1, cos_sin_rows=40,
+                              k_scale=0.05, v_scale=0.05)
+    r, _ = run_and_check(w)
+    assert (r.flags.cpu().numpy() == 0).all()
+
+
+BAD = {
+    "first_nonzero": dict(q_indptr=[1, 2, 2, 5]),
+    "non_monotone": dict(q_indptr=[0, 3, 2, 5]),
+    "last_short": dict(q_indptr=[0, 2, 2, 4]),
+    "last_long": dict(q_indptr=[0, 2, 2, 6]),
+    "seq_shorter_than_new": dict(seq_lens=[5, 4, 2]),
+    "negative_seq_len": dict(seq_lens=[5, -1, 3]),
+    "page_table_overrun": dict(seq_lens=[13, 4, 3]),
+    "cos_sin_overrun": dict(seq_lens=[5, 4, 12]),
+}
+
+
+@pytest.mark.parametrize("case", sorted(BAD))
+@pytest.mark.parametrize("policy", [0, 1, 2])
+def test_each_malformed_predicate_writes_nothing(case, policy):
+    w = workloads.make_append(seed=4, n_new=[2, 0, 3], seq_lens=[5, 4, 3], Hq=4, Hkv=2,
+                              page_size=4, max_pages=3, quant_policy=policy, cos_sin_rows=11,
+                              k_scale=0.05, v_scale=0.05, q_scale_inv=20.0)
+    over = {k: np.array(v, np.int32) for k, v in BAD[case].items()}
+    r = AppendRun(w, **over)
+    r.launch()
+    assert r.check() == {"flagged": True}
+    assert (r.flags.cpu().numpy() == -1).all()
+
+
+@pytest.mark.parametrize("bad", [-1, 11])
+def test_explicit_position_out_of_range_writes_nothing(bad):
+    w = workloads.make_append(seed=5, n_new=[2, 3], seq_lens=[2, 3], Hq=4, Hkv=2, page_size=4,
+                              max_pages=2, cos_sin_rows=11, positions=[0, 1, 2, bad, 4])
+    r = AppendRun(w)
+    r.launch()
+    assert r.check() == {"flagged": True}
+
+
+def test_largest_batch():
+    B = 16384
+    rng = np.random.default_rng(8)
+    L = rng.integers(1, 64, B)
+    w = workloads.make_append(seed=8, n_new=[1] * B, seq_lens=L, Hq=2, Hkv=1, page_size=16,
+                              max_pages=4, quant_policy=1, cos_sin_rows=64, k_scale=0.05,
+                              v_scale=0.05)
+    run_and_check(w)
+
+
+def test_padded_page_stride():
+    w = workloads.make_append(seed=9, n_new=[5, 17, 0, 1], seq_lens=[9, 30, 7, 1], Hq=8,
+                              Hkv=2, page_size=16, max_pages=3, quant_policy=2,
+                              q_scale_inv=20.0, k_scale=0.05, v_scale=0.05)
+    run_and_check(w, page_stride_pad=256)
+
+
+def test_every_bf16_input_through_the_fp8_encoder():
+    """All 65536 BF16 codes (inf and NaN included) as Q inputs with no norm and
+    an identity rotation (GPT-J, rot_dim 2, position 0), static scale 1: the
+    payload is the E4M3 encoding of the input itself, and the GPU's packed
+    conversion must equal the oracle's encoder on every code."""
+    Hq, Hkv = 8, 1
+    per_head = D - 2
+    heads = -(-65536 // per_head)
+    T = -(-heads // Hq)
+    w = workloads.make_append(seed=10, n_new=[1] * T, seq_lens=[1] * T, Hq=Hq, Hkv=Hkv,
+                              page_size=4, max_pages=1, quant_policy=2, norm=False, rot_dim=2,
+                              rope_style=1, q_scale_inv=1.0, k_scale=1.0, v_scale=1.0)
+    codes = np.zeros(T * Hq * per_head, np.uint16)
+    codes[:65536] = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    q = w.qkv[:, : Hq * D].reshape(T, Hq, D)
+    q[:, :, 2:] = codes.reshape(T, Hq, per_head)
+    q[:, :, :2] = 0x3F80                      # the rotated pair stays finite
+    w.qkv[:, : Hq * D] = q.reshape(T, Hq * D)
+    r, rep = run_and_check(w)
+    assert rep["q_exact_frac"] == 1.0
+    # the payload is the encoding of the input value itself (NaN codes equal)
+    got = _np(r.out_q).reshape(T, Hq, D)[:, :, 2:].reshape(-1)[:65536]
+    want = oracle.e4m3(bf16_bits_to_f32(codes[:65536]))
+    assert (ulp_e4m3(got, want) == 0).all()
+
+
+def test_heads_far_apart_in_scale_normalise_independently():
+    w = workloads.make_append(seed=12, n_new=[3, 2], seq_lens=[40, 2], Hq=16, Hkv=4,
+                              page_size=16, max_pages=3, quant_policy=0)
+    x = bf16_bits_to_f32(w.qkv).copy()
+    for h in range(0, 24, 2):
+        x[:, h * D:(h + 1) * D] *= 1e3
+    w.qkv = (x.view(np.uint32) >> 16).astype(np.uint16)
+    run_and_check(w)
+
+
+def test_non_default_stream():
+    w = workloads.tiny_decode_bf16()
+    r = AppendRun(w)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        r.launch(stream=s)
+    s.synchronize()
+    r.check()
+
+
+def test_cuda_graph_capture_and_replay_is_bitwise_eager():
+    w = workloads.fp8_decode_dynamic()
+    r = AppendRun(w)
+    r.launch()
+    torch.cuda.synchronize()
+    eager = (r.out_q.clone(), r.q_scale.clone(), r.k_store.clone(), r.v_store.clone(),
+             r.flags.clone())
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        r.launch(stream=s)
+    for _ in range(3):
+        r.out_q.fill_(0x55)
+        r.q_scale.fill_(-1.0)
+        r.flags.fill_(7)
+        g.replay()
+        torch.cuda.synchronize()
+        now = (r.out_q, r.q_scale, r.k_store, r.v_store, r.flags)
+        for a, b in zip(eager, now):
+            assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    del g
+    r.check()

@@ -15,6 +15,7 @@ page tables; the vLLM issue #24678 model table for the DeepSeek-R1 MLA shape).
 """
 from __future__ import annotations
 
+import functools
 from dataclasses import dataclass, field
 from typing import Optional
 
@@ -38,7 +39,12 @@ def cos_sin_cache(rows: int, rot: int, theta: float) -> np.ndarray:
     """fp32 [rows, rot] = [cos(p * f_i) | sin(p * f_i)], f_i = theta^(-2i/rot).
 
     Tabulated in float64 and rounded once to float32; row 0 is exactly
-    [1, ..., 1 | 0, ..., 0]."""
+    [1, ..., 1 | 0, ..., 0].  Returns a fresh copy (tables are memoised)."""
+    return _cos_sin_cache(int(rows), int(rot), float(theta)).copy()
+
+
+@functools.lru_cache(maxsize=16)
+def _cos_sin_cache(rows: int, rot: int, theta: float) -> np.ndarray:
     half = rot // 2
     inv_freq = theta ** (-(np.arange(half, dtype=np.float64) * 2.0) / rot)
     ang = np.arange(rows, dtype=np.float64)[:, None] * inv_freq[None, :]
