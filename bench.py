@@ -58,11 +58,16 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=2000)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=MAIN_WORKLOAD, choices=sorted(workloads.APPEND_CONFIGS))
+    ap.add_argument("--replicas", type=int, default=None, help="override the replica count")
     ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU budget of the oracle baseline sample")
     ap.add_argument("--e2e-steps", type=int, default=3000)
+    ap.add_argument("--profile", action="store_true",
+                    help="profiling run: only --workload (or mla_decode), --steps eager launches, "
+                         "no graphs, no e2e / per-config / CPU legs, no JSON line")
+    ap.add_argument("--mla", action="store_true", help="with --profile: the MLA workload")
     return ap.parse_args(argv)
 
 
@@ -516,6 +521,8 @@ def main(argv=None):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.profile:
+        return run_profile(args, torch, fqr, dev)
     dist = None
     if world > 1:
         import datetime
@@ -570,6 +577,23 @@ def main(argv=None):
         "per_config": per_config,
     }
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_profile(args, torch, fqr, dev):
+    """A few eager launches of one workload for ncu (small device footprint)."""
+    if args.mla:
+        b = MlaBench(torch, fqr, dev, max_replicas=args.replicas or 2)
+    else:
+        b = AppendBench(args.workload, torch, fqr, dev, max_replicas=args.replicas or 2)
+    h = torch.cuda.current_stream().cuda_stream
+    for i in range(args.warmup + args.steps):
+        b.launch(i, h)
+    torch.cuda.synchronize()
+    if not args.mla:
+        b.check_flags()
+    print(f"profile: {b.name} x {args.warmup + args.steps} launches, {b.R} replicas, "
+          f"{max(b.bytes) / 1e6:.1f} MB per launch")
     return 0
 
 

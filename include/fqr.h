@@ -120,7 +120,7 @@ typedef struct fqr_append_params {
    * elements apart (>= page_size * Hkv * 128, 16-byte multiples). */
   void* k_cache;
   void* v_cache;
-  int32_t num_pages, page_size;
+  int32_t num_pages, page_size;  /* 2 * B * (page_size - 1) < 2^31              */
   int64_t k_page_stride, v_page_stride;
   int32_t quant_policy;       /* 0, 1 or 2, see above                         */
   const float* q_scale_inv;   /* device fp32 scalar (policy 2)                */

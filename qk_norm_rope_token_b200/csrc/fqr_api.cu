@@ -30,6 +30,8 @@ int check_append(const fqr_append_params* p) {
     return FQR_EINVAL;
   if (p->page_size <= 0 || p->num_pages <= 0 || p->max_pages <= 0 || p->cos_sin_rows <= 0)
     return FQR_EINVAL;
+  // tail rows of the whole batch are counted in 32 bits
+  if (2 * static_cast<int64_t>(p->B) * (p->page_size - 1) >= (int64_t{1} << 31)) return FQR_EINVAL;
   const int64_t H = static_cast<int64_t>(p->Hq) + 2 * static_cast<int64_t>(p->Hkv);
   if (p->qkv_row_stride < H * FQR_HEAD_DIM || p->qkv_row_stride % 8 != 0) return FQR_EINVAL;
   const int64_t esize = p->quant_policy == 0 ? 2 : 1;

@@ -90,6 +90,7 @@ APPEND_BAD = {
     "tokens_without_requests": dict(B=0),
     "page_size_zero": dict(page_size=0),
     "page_size_negative": dict(page_size=-4),
+    "tail_rows_overflow": dict(B=16384, page_size=65537),
     "policy_3": dict(quant_policy=3),
     "rope_style_2": dict(rope_style=2),
     "rot_odd": dict(rope_style=1, rot_dim=63),
