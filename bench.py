@@ -59,6 +59,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=MAIN_WORKLOAD, choices=sorted(workloads.APPEND_CONFIGS))
     ap.add_argument("--replicas", type=int, default=None, help="override the replica count")
+    ap.add_argument("--schedule", type=int, default=0, choices=[0, 1, 2],
+                    help="0 automatic, 1 latency, 2 streaming")
     ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -185,8 +187,9 @@ class AppendBench:
     """R replicas of one append workload sharing one pair of KV caches."""
 
     def __init__(self, name, torch, fqr, device, min_bytes=3 * L2_BYTES, max_replicas=64,
-                 seed_offset=0):
+                 seed_offset=0, schedule=0):
         self.torch, self.fqr, self.dev = torch, fqr, device
+        self.schedule = schedule
         base = workloads.APPEND_CONFIGS[name]()
         self.name = base.name
         per = workloads.append_bytes(base)["total"]
@@ -237,7 +240,7 @@ class AppendBench:
                     q_scale_inv=self.scales["q_scale_inv"] if w.quant_policy == 2 else None,
                     k_scale=self.scales["k_scale"] if w.quant_policy else None,
                     v_scale=self.scales["v_scale"] if w.quant_policy else None,
-                    upper_max=w.upper_max)
+                    upper_max=w.upper_max, schedule=self.schedule)
 
     def _params(self, w, st):
         return self.fqr.append_params(st["qkv"], self.cs, st["q_indptr"], st["seq_lens"],
@@ -535,7 +538,8 @@ def main(argv=None):
             dist.barrier()
 
     peak, peak_src = load_peaks()
-    bench = AppendBench(args.workload, torch, fqr, dev, seed_offset=1000 * rank)
+    bench = AppendBench(args.workload, torch, fqr, dev, seed_offset=1000 * rank,
+                        schedule=args.schedule)
     sampler = ClockSampler(gpu_smi_id(torch, dev)) if rank == 0 else None
     if sampler is not None:
         time.sleep(1.0)   # let nvidia-smi start sampling before the warm-up
@@ -585,7 +589,8 @@ def run_profile(args, torch, fqr, dev):
     if args.mla:
         b = MlaBench(torch, fqr, dev, max_replicas=args.replicas or 2)
     else:
-        b = AppendBench(args.workload, torch, fqr, dev, max_replicas=args.replicas or 2)
+        b = AppendBench(args.workload, torch, fqr, dev, max_replicas=args.replicas or 2,
+                        schedule=args.schedule)
     h = torch.cuda.current_stream().cuda_stream
     for i in range(args.warmup + args.steps):
         b.launch(i, h)
@@ -608,7 +613,13 @@ def measure_per_config(torch, fqr, dev, peak, main_name, steps=20000, warmup=200
         gbs = nbytes / n / (us * 1e-6) / 1e9
         out[name] = {"workload": b.name, "us_per_launch": us, "tokens_per_s": b.T / (us * 1e-6),
                      "GB_per_s": gbs, "frac_of_peak": gbs / peak,
-                     "bytes_per_launch": nbytes / n, "replicas": b.R, "launches": n}
+                     "bytes_per_launch": nbytes / n, "replicas": b.R, "launches": n,
+                     "us_per_launch_by_schedule": {}}
+        for sched, label in ((1, "latency"), (2, "streaming")):   # both schedules, for tuning
+            for st in b.reps:
+                st["params"].schedule = sched
+            ms_s, _ = time_launches(torch, b, n, warmup)
+            out[name]["us_per_launch_by_schedule"][label] = ms_s * 1e3 / n
         del b
         torch.cuda.empty_cache()
     m = MlaBench(torch, fqr, dev)

@@ -40,6 +40,13 @@ extern "C" {
 #define FQR_ECUDA 3
 
 #define FQR_HEAD_DIM 128
+
+/* fqr_append_params.schedule: how rows are spread over the GPU (the results
+ * are identical).  AUTO picks LATENCY for small batches (decode) and
+ * STREAMING for large ones (prefill). */
+#define FQR_SCHEDULE_AUTO 0
+#define FQR_SCHEDULE_LATENCY 1
+#define FQR_SCHEDULE_STREAMING 2
 /* Largest batch (number of requests) one call accepts; per-request metadata
  * is staged in shared memory by every thread block. */
 #define FQR_MAX_BATCH 16384
@@ -76,6 +83,8 @@ extern "C" {
  * page_table[b, (L_b-1) / P] are zeroed in both caches.
  *
  * flags[b] = 0 after a valid call (requests without new tokens included).
+ * flags[b] = -2 (all flags) only if the kernel gave up waiting for its own
+ * shared-memory copies (a bounded wait that should never expire).
  * If the metadata is malformed -- q_indptr[0] != 0, q_indptr[B] != T, any
  * q_indptr decrease, L_b < n_b, L_b > max_pages * P, or (derived positions)
  * L_b > cos_sin_rows, or (explicit positions) any position outside
@@ -132,6 +141,7 @@ typedef struct fqr_append_params {
   void* out_q;
   float* q_scale;
   int32_t* flags;
+  int32_t schedule;           /* FQR_SCHEDULE_*; 0 = automatic                */
 } fqr_append_params;
 
 int fqr_append_paged(const fqr_append_params* p, void* stream);

@@ -21,6 +21,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfqr.so")
 
 FQR_OK, FQR_EINVAL, FQR_ENOTSUP, FQR_ECUDA = 0, 1, 2, 3
+SCHEDULE_AUTO, SCHEDULE_LATENCY, SCHEDULE_STREAMING = 0, 1, 2
+FLAG_TIMEOUT = -2
 HEAD_DIM = 128
 MAX_BATCH = 16384
 
@@ -40,7 +42,7 @@ class AppendParams(ctypes.Structure):
         ("k_page_stride", c_i64), ("v_page_stride", c_i64),
         ("quant_policy", c_i32),
         ("q_scale_inv", c_vp), ("k_scale", c_vp), ("v_scale", c_vp), ("upper_max", c_f32),
-        ("out_q", c_vp), ("q_scale", c_vp), ("flags", c_vp),
+        ("out_q", c_vp), ("q_scale", c_vp), ("flags", c_vp), ("schedule", c_i32),
     ]
 
 
@@ -111,7 +113,8 @@ def append_params(qkv, cos_sin_cache, q_indptr, seq_lens, page_table, k_cache, v
                   out_q, flags, *, q_norm_w=None, k_norm_w=None, eps: float = 1e-6,
                   positions=None, rope_style: int = 0, rot_dim: Optional[int] = None,
                   quant_policy: int = 0, q_scale=None, q_scale_inv=None, k_scale=None,
-                  v_scale=None, upper_max: float = 448.0) -> AppendParams:
+                  v_scale=None, upper_max: float = 448.0,
+                  schedule: int = SCHEDULE_AUTO) -> AppendParams:
     """Fill an AppendParams from tensors (shapes as in include/fqr.h)."""
     T = int(qkv.shape[0])
     return AppendParams(
@@ -129,7 +132,7 @@ def append_params(qkv, cos_sin_cache, q_indptr, seq_lens, page_table, k_cache, v
         k_page_stride=int(k_cache.stride(0)), v_page_stride=int(v_cache.stride(0)),
         quant_policy=int(quant_policy), q_scale_inv=_ptr(q_scale_inv),
         k_scale=_ptr(k_scale), v_scale=_ptr(v_scale), upper_max=float(upper_max),
-        out_q=_ptr(out_q), q_scale=_ptr(q_scale), flags=_ptr(flags))
+        out_q=_ptr(out_q), q_scale=_ptr(q_scale), flags=_ptr(flags), schedule=int(schedule))
 
 
 def append_paged(qkv, cos_sin_cache, q_indptr, seq_lens, page_table, k_cache, v_cache,
@@ -210,4 +213,5 @@ __all__ = ["LIB", "LIB_PATH", "AppendParams", "MlaParams", "FqrError", "strerror
            "append_paged_from_host",
            "append_params", "append_paged", "append_paged_raw", "mla_params",
            "concat_mla_cache", "concat_mla_cache_raw", "FQR_OK", "FQR_EINVAL",
-           "FQR_ENOTSUP", "FQR_ECUDA", "HEAD_DIM", "MAX_BATCH"]
+           "FQR_ENOTSUP", "FQR_ECUDA", "HEAD_DIM", "MAX_BATCH", "SCHEDULE_AUTO",
+           "SCHEDULE_LATENCY", "SCHEDULE_STREAMING", "FLAG_TIMEOUT"]

@@ -56,6 +56,7 @@ int check_append(const fqr_append_params* p) {
   if (p->quant_policy == 1 && (!p->q_scale || !aligned(p->q_scale, 4))) return FQR_EINVAL;
   if (p->quant_policy == 2 && !p->q_scale_inv) return FQR_EINVAL;
   if (p->quant_policy != 0 && (!p->k_scale || !p->v_scale)) return FQR_EINVAL;
+  if (p->schedule < FQR_SCHEDULE_AUTO || p->schedule > FQR_SCHEDULE_STREAMING) return FQR_EINVAL;
   if (p->rope_style == 0 && p->rot_dim != FQR_HEAD_DIM) return FQR_ENOTSUP;
   return FQR_OK;
 }

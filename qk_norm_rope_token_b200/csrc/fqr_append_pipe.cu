@@ -1,0 +1,365 @@
+// fqr_append_pipe.cu -- streaming schedule of the fused append (large
+// batches, e.g. prefill): each block pipelines its rows through shared memory.
+//
+// Method: FlashInfer PR #5956, section "Contract" (see fqr_head.cuh for the
+// per-head arithmetic).
+//
+// One block = 1 producer warp + 8 consumer warps; persistent grid, every
+// block resident; each block owns a contiguous range of units (a unit is one
+// packed row, or a chunk of its heads for very wide rows).
+//   * the producer streams each unit into a ring of shared-memory stages with
+//     1-D bulk copies (cp.async.bulk, the TMA engine; never multicast): the
+//     packed heads and the token's cos/sin row, completing on a "full"
+//     mbarrier.  The first stages' packed heads are requested before the
+//     validation prologue.  The producer's 32 lanes resolve request, position
+//     and page id of 32 units in parallel; the cos/sin copy is issued before
+//     the page id is known, and the stage header (slot, page, position, last
+//     row) is published by the arrive that completes the phase.
+//   * consumer warps take 4 heads at a time from the stage (fqr_head.cuh),
+//     store straight to out_q / the cache slot and release the stage on its
+//     "empty" mbarrier; the quad -> warp assignment rotates every unit.
+//   * the K/V heads of a request's last row zero their column of the tail
+//     rows; consumer warps of the grid zero the tails of requests that append
+//     nothing.
+//   * every block validates the whole batch first; every wait is bounded
+//     (kWaitLimitNs) and a wait that gives up sets every flag to kFlagTimeout.
+#include "fqr_head.cuh"
+#include "fqr_launch.h"
+
+namespace fqr {
+
+constexpr int kConsumers = 8;
+constexpr int kPipeThreads = (kConsumers + 1) * 32;
+constexpr int kMaxStages = 8;
+constexpr int kFixedSmem = 1280;  // barriers (128) + fp32 weights (1024) + spare
+
+// Stage header, written by the producer before it arrives on "full".
+struct StageInfo {
+  int p_slot, page, pos, is_last;
+};
+
+struct PipeArgs {
+  HeadParams hp;
+  const uint16_t* qkv;
+  int64_t row_stride;
+  int T, B, H;
+  int chunk_heads, nchunks;
+  int64_t units;
+  const uint16_t* qw;
+  const uint16_t* kw;
+  const float* cs;
+  int cs_rows, cs_bulk, cs_bytes;
+  const int64_t* positions;
+  const int32_t* q_indptr;
+  const int32_t* seq_lens;
+  const int32_t* page_table;
+  int max_pages;
+  int32_t* flags;
+  int stages, stage_bytes;
+};
+
+__device__ __forceinline__ uint4 ld_smem_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(smem_addr(p)));
+  return r;
+}
+__device__ __forceinline__ float4 ld_smem_f4(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+
+__device__ void report_timeout(const PipeArgs& a) {
+  for (int b = threadIdx.x & 31; b < a.B; b += 32) a.flags[b] = kFlagTimeout;
+}
+
+// Unit u: packed row t, heads [h0, h0 + nh).
+__device__ __forceinline__ void unit_heads(const PipeArgs& a, int64_t u, int& t, int& h0,
+                                           int& nh) {
+  t = static_cast<int>(u / a.nchunks);
+  h0 = static_cast<int>(u - static_cast<int64_t>(t) * a.nchunks) * a.chunk_heads;
+  nh = min(a.H - h0, a.chunk_heads);
+}
+
+// Producer lane: bulk-copy the packed heads of unit u into stage `st`.
+__device__ __forceinline__ void issue_heads(const PipeArgs& a, unsigned char* st, int64_t u,
+                                            uint64_t* bar) {
+  int t, h0, nh;
+  unit_heads(a, u, t, h0, nh);
+  const uint32_t bytes = static_cast<uint32_t>(nh) * kHeadDim * 2;
+  mbar_expect_tx(bar, bytes);
+  bulk_g2s(st + 16 + a.cs_bytes,
+           a.qkv + static_cast<int64_t>(t) * a.row_stride + static_cast<int64_t>(h0) * kHeadDim,
+           bytes, bar);
+}
+
+// ------------------------------------------------------------- producer --
+__device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full,
+                        uint64_t* empty, const int* s_indptr, const int* s_seq, int64_t u0,
+                        int nunits, int pre) {
+  const int lane = threadIdx.x & 31;
+  const int S = a.stages;
+  int ok = 1;
+  int issued = pre;  // stages whose head copies are in flight or consumed
+  for (int i0 = 0; i0 < nunits && ok; i0 += 32) {
+    // lane j prepares unit i0 + j in parallel with the others
+    StageInfo info{0, 0, 0, 0};  // p_slot, page, pos, is_last
+    int need_cs = 0;
+    if (i0 + lane < nunits) {
+      int t, h0, nh;
+      unit_heads(a, u0 + i0 + lane, t, h0, nh);
+      const int b = request_of_row(s_indptr, a.B, t);
+      const int end = s_indptr[b + 1];
+      const int p = t + s_seq[b] - end;
+      info.p_slot = p;
+      info.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : p;
+      info.is_last = t == end - 1;
+      if (h0 + nh > a.hp.Hq)  // the unit holds K or V heads: it needs the page id
+        info.page =
+            __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + p / a.hp.page_size);
+      need_cs = (h0 < a.hp.Hq + a.hp.Hkv) && a.cs_bulk;
+    }
+    const int n = min(32, nunits - i0);
+    for (int j = 0; j < n; ++j) {
+      // position first: the cos/sin copy must not wait for the page-id load
+      const int posj = __shfl_sync(0xffffffffu, info.pos, j);
+      const int csj = __shfl_sync(0xffffffffu, need_cs, j);
+      const int i = i0 + j, s = i % S;
+      uint64_t* fb = &full[s];
+      unsigned char* st = stages + static_cast<size_t>(s) * a.stage_bytes;
+      if (lane == 0) {
+        if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1)) ok = 0;
+        if (ok) {
+          fence_proxy_async_smem();
+          if (i >= pre) {
+            issue_heads(a, st, u0 + i, fb);
+            ++issued;
+          }
+          if (csj) {
+            const uint32_t cb = static_cast<uint32_t>(a.hp.rot) * 4;
+            mbar_expect_tx(fb, cb);
+            bulk_g2s(st + 16, a.cs + static_cast<int64_t>(posj) * a.hp.rot, cb, fb);
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const StageInfo sj{__shfl_sync(0xffffffffu, info.p_slot, j),
+                         __shfl_sync(0xffffffffu, info.page, j), posj,
+                         __shfl_sync(0xffffffffu, info.is_last, j)};
+      if (lane == 0) {
+        *reinterpret_cast<StageInfo*>(st) = sj;
+        mbar_arrive(fb);  // release: the header is visible once the phase completes
+      }
+    }
+  }
+  if (!ok) {
+    report_timeout(a);
+    if (lane == 0) {  // let the copies already issued land before the block leaves
+      const int first = issued > S ? issued - S : 0;
+      for (int i = first; i < issued; ++i) mbar_wait(&full[i % S], (i / S) & 1);
+    }
+  }
+}
+
+// ------------------------------------------------------------ consumers --
+template <int POLICY, int STYLE>
+__device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t* full,
+                        uint64_t* empty, const float* s_w, int64_t u0, int nunits) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 3, l8 = lane & 7;
+  const unsigned gmask = 0xFFu << (8 * g);
+  const int S = a.stages;
+  // (row, chunk) of the current unit, advanced without dividing
+  int t = static_cast<int>(u0 / a.nchunks);
+  int c = static_cast<int>(u0 - static_cast<int64_t>(t) * a.nchunks);
+  int rot = 0;  // quad -> warp rotation, advanced by nq every unit
+  for (int i = 0; i < nunits; ++i) {
+    const int s = i % S;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / S) & 1))) {
+      report_timeout(a);
+      return;
+    }
+    const unsigned char* st = stages + static_cast<size_t>(s) * a.stage_bytes;
+    const StageInfo info = *reinterpret_cast<const StageInfo*>(st);
+    const RowCtx r{t, info.p_slot, info.pos, info.page, info.is_last};
+    const float* cs_row = a.cs_bulk ? reinterpret_cast<const float*>(st + 16)
+                                    : a.cs + static_cast<int64_t>(info.pos) * a.hp.rot;
+    const int h0 = c * a.chunk_heads, nh = min(a.H - h0, a.chunk_heads);
+    const int nq = (nh + 3) >> 2;
+    int q = warp - rot;
+    if (q < 0) q += kConsumers;
+    for (; q < nq; q += kConsumers) {
+      const int hl = 4 * q + g;
+      if (hl < nh) {
+        const unsigned char* src = st + 16 + a.cs_bytes + hl * (kHeadDim * 2) + 16 * l8;
+        process_head<POLICY, STYLE>(a.hp, r, h0 + hl, ld_smem_v4(src), ld_smem_v4(src + 128),
+                                    cs_row, s_w, l8, gmask);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    rot = (rot + nq) & (kConsumers - 1);
+    if (++c == a.nchunks) {
+      c = 0;
+      ++t;
+    }
+  }
+}
+
+// Tails of requests that append no row in this call, spread over every
+// consumer warp of the grid.
+template <int POLICY>
+__device__ void zero_empty_request_tails(const PipeArgs& a, const int* s_indptr, const int* s_seq) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int W = gridDim.x * kConsumers;
+  for (int b = blockIdx.x * kConsumers + warp; b < a.B; b += W) {
+    const int L = s_seq[b];
+    if (s_indptr[b] == s_indptr[b + 1] && L > 0)
+      zero_request_tail<POLICY == 0 ? 2 : 1>(a.hp, a.page_table, a.max_pages, b, L, lane);
+  }
+}
+
+template <int POLICY, int STYLE>
+__global__ void __launch_bounds__(kPipeThreads) pipe_append_kernel(const PipeArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kMaxStages;
+  float* s_w = reinterpret_cast<float*>(smem + 128);   // staged fp32 weights (fqr_head.cuh)
+  unsigned char* stages = smem + kFixedSmem;
+  int* s_indptr = reinterpret_cast<int*>(stages + static_cast<size_t>(a.stages) * a.stage_bytes);
+  int* s_seq = s_indptr + a.B + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool producer = warp == kConsumers;
+  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * a.units / gridDim.x;
+  const int64_t u1 = static_cast<int64_t>(blockIdx.x + 1) * a.units / gridDim.x;
+  const int nunits = static_cast<int>(u1 - u0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers);
+    }
+    mbar_init_fence();
+  }
+  // Programmatic dependent launch: everything above touched only shared
+  // memory; wait for the preceding grid before reading any input, and let the
+  // next grid in the stream start its own set-up early.
+  grid_dependency_wait();
+  grid_launch_dependents();
+  __syncthreads();
+
+  // The first stages' packed heads need no metadata: start them now so their
+  // latency overlaps the validation prologue.
+  int pre = 0;
+  if (producer && lane == 0) {
+    pre = min(a.stages, nunits);
+    for (int i = 0; i < pre; ++i)
+      issue_heads(a, stages + static_cast<size_t>(i) * a.stage_bytes, u0 + i, &full[i]);
+  }
+  stage_weights(s_w, a.qw, a.kw);
+
+  const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
+               static_cast<int64_t>(a.max_pages) * a.hp.page_size, a.cs_rows};
+  if (stage_and_validate(m, s_indptr, s_seq)) {
+    if (producer && lane == 0) {  // drain the copies issued before the verdict
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive(&full[i]);
+        mbar_wait(&full[i], 0);
+      }
+    }
+    return;
+  }
+
+  if (producer) {
+    produce(a, stages, full, empty, s_indptr, s_seq, u0, nunits, pre);
+  } else {
+    zero_empty_request_tails<POLICY>(a, s_indptr, s_seq);
+    consume<POLICY, STYLE>(a, stages, full, empty, s_w, u0, nunits);
+  }
+}
+
+using PipeKernel = void (*)(const PipeArgs);
+
+static PipeKernel select_pipe(int policy, int style) {
+  if (style == 0) {
+    if (policy == 0) return pipe_append_kernel<0, 0>;
+    if (policy == 1) return pipe_append_kernel<1, 0>;
+    return pipe_append_kernel<2, 0>;
+  }
+  if (policy == 0) return pipe_append_kernel<0, 1>;
+  if (policy == 1) return pipe_append_kernel<1, 1>;
+  return pipe_append_kernel<2, 1>;
+}
+
+int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream) {
+  PipeArgs a;
+  a.hp = hp;
+  a.qkv = p.qkv;
+  a.row_stride = p.qkv_row_stride;
+  a.T = p.T;
+  a.B = p.B;
+  a.H = p.Hq + 2 * p.Hkv;
+  a.qw = p.q_norm_w;
+  a.kw = p.k_norm_w;
+  a.cs = p.cos_sin_cache;
+  a.cs_rows = p.cos_sin_rows;
+  a.cs_bulk = (p.rot_dim * 4) % 16 == 0 ? 1 : 0;
+  a.cs_bytes = a.cs_bulk ? p.rot_dim * 4 : 0;
+  a.positions = p.positions;
+  a.q_indptr = p.q_indptr;
+  a.seq_lens = p.seq_lens;
+  a.page_table = p.page_table;
+  a.max_pages = p.max_pages;
+  a.flags = p.flags;
+
+  int dev = 0, sms = 0, smem_optin = 0, smem_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+          cudaSuccess)
+    return FQR_ECUDA;
+
+  const int64_t meta = static_cast<int64_t>(2 * p.B + 1) * sizeof(int);
+  auto stage_bytes = [&](int hc) { return 16 + a.cs_bytes + hc * kHeadDim * 2; };
+  // a row that does not fit two stages beside the metadata is split into
+  // chunks of whole quads
+  int hc = a.H;
+  while (hc > 4 && kFixedSmem + meta + 2 * stage_bytes(hc) > smem_optin) hc = ((hc / 2 + 3) / 4) * 4;
+  if (kFixedSmem + meta + stage_bytes(hc) > smem_optin) return FQR_ENOTSUP;
+  a.chunk_heads = hc;
+  a.nchunks = (a.H + hc - 1) / hc;
+  a.units = static_cast<int64_t>(p.T) * a.nchunks;
+  a.stage_bytes = stage_bytes(hc);
+  // pipeline depth: aim at two resident blocks per SM, never deeper than the
+  // units a block will see
+  const int64_t per_block_budget = smem_sm / 2 - 1024;
+  int S = static_cast<int>((per_block_budget - kFixedSmem - meta) / a.stage_bytes);
+  S = S < 1 ? 1 : (S > kMaxStages ? kMaxStages : S);
+  const int64_t upb = (a.units + 2 * sms - 1) / (2 * sms);
+  if (upb >= 1 && S > upb) S = static_cast<int>(upb);
+  while (S > 1 && kFixedSmem + meta + static_cast<int64_t>(S) * a.stage_bytes > smem_optin) --S;
+  a.stages = S;
+  const size_t smem = static_cast<size_t>(kFixedSmem + meta + static_cast<int64_t>(S) * a.stage_bytes);
+
+  PipeKernel k = select_pipe(p.quant_policy, p.rope_style);
+  const void* fn = reinterpret_cast<const void*>(k);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return FQR_ECUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kPipeThreads, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return FQR_ECUDA;
+  const int64_t cap = static_cast<int64_t>(per_sm) * sms;
+  const int64_t want = a.units > sms ? a.units : sms;
+  const int grid = static_cast<int>(want < cap ? want : cap);
+  return launch_pdl(k, grid, kPipeThreads, smem, stream, a);
+}
+
+}  // namespace fqr

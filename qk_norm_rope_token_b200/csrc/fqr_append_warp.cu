@@ -1,0 +1,143 @@
+// fqr_append_warp.cu -- latency schedule of the fused append (small batches,
+// e.g. decode): many independent warp tasks, all resident at once.
+//
+// Method: FlashInfer PR #5956, section "Contract" (see fqr_head.cuh for the
+// per-head arithmetic).
+//
+//   * head task = 4 heads of one packed row (8 lanes per head); the task's two
+//     16-byte loads per lane need no metadata and are issued before the
+//     validation prologue; the next task's loads are issued before the current
+//     task is computed.
+//   * every block stages q_indptr / seq_lens in shared memory and validates the
+//     whole batch (stage_and_validate); a malformed batch writes only flags.
+//   * the K/V heads of a request's last new row also zero their column of the
+//     tail rows of that page; one "request task" per request zeroes the tail of
+//     requests that append nothing in this call.
+#include "fqr_head.cuh"
+#include "fqr_launch.h"
+
+namespace fqr {
+
+struct WarpArgs {
+  HeadParams hp;
+  const uint16_t* qkv;
+  int64_t row_stride;
+  int T, B, H, quads, n_head;
+  const uint16_t* qw;
+  const uint16_t* kw;
+  const float* cs;
+  int cs_rows;
+  const int64_t* positions;
+  const int32_t* q_indptr;
+  const int32_t* seq_lens;
+  const int32_t* page_table;
+  int max_pages;
+  int32_t* flags;
+};
+
+__device__ __forceinline__ void warp_load_head(const WarpArgs& a, int w, int g, int l8, uint4& xa,
+                                               uint4& xb) {
+  const int t = w / a.quads;
+  const int h = (w - t * a.quads) * 4 + g;
+  if (h < a.H) {
+    const uint16_t* src = a.qkv + static_cast<int64_t>(t) * a.row_stride + h * kHeadDim + 8 * l8;
+    xa = ld_stream_v4(src);
+    xb = ld_stream_v4(src + 64);
+  }
+}
+
+template <int POLICY, int STYLE>
+__global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a) {
+  extern __shared__ __align__(16) int smem[];
+  float* s_w = reinterpret_cast<float*>(smem);  // 256 fp32 weights
+  int* s_indptr = smem + 2 * kHeadDim;          // B + 1
+  int* s_seq = s_indptr + a.B + 1;              // B
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 3, l8 = lane & 7;
+  const unsigned gmask = 0xFFu << (8 * g);
+  const int gwarp = blockIdx.x * kWarps + warp;
+  const int nwarps = gridDim.x * kWarps;
+
+  grid_dependency_wait();
+  grid_launch_dependents();
+
+  uint4 pa = make_uint4(0u, 0u, 0u, 0u), pb = pa;
+  if (gwarp < a.n_head) warp_load_head(a, gwarp, g, l8, pa, pb);
+  stage_weights(s_w, a.qw, a.kw);
+
+  const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
+               static_cast<int64_t>(a.max_pages) * a.hp.page_size, a.cs_rows};
+  if (stage_and_validate(m, s_indptr, s_seq)) return;
+
+  const int n_tasks = a.n_head + a.B;
+  for (int w = gwarp; w < n_tasks; w += nwarps) {
+    if (w < a.n_head) {
+      const uint4 xa = pa, xb = pb;
+      if (w + nwarps < a.n_head) warp_load_head(a, w + nwarps, g, l8, pa, pb);
+      const int t = w / a.quads;
+      const int h = (w - t * a.quads) * 4 + g;
+      if (h >= a.H) continue;  // the whole 8-lane group skips together
+      const int b = request_of_row(s_indptr, a.B, t);
+      const int end = s_indptr[b + 1];
+      RowCtx r;
+      r.t = t;
+      r.p_slot = t + s_seq[b] - end;
+      r.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : r.p_slot;
+      r.is_last = t == end - 1;
+      r.page = h >= a.hp.Hq
+                   ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + r.p_slot / a.hp.page_size)
+                   : 0;
+      const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
+      process_head<POLICY, STYLE>(a.hp, r, h, xa, xb, cs_row, s_w, l8, gmask);
+    } else {
+      const int b = w - a.n_head;  // request task: tail of a request without new rows
+      const int L = s_seq[b];
+      if (s_indptr[b] == s_indptr[b + 1] && L > 0)
+        zero_request_tail<POLICY == 0 ? 2 : 1>(a.hp, a.page_table, a.max_pages, b, L, lane);
+    }
+  }
+}
+
+using WarpKernel = void (*)(const WarpArgs);
+
+static WarpKernel select_warp(int policy, int style) {
+  if (style == 0) {
+    if (policy == 0) return warp_append_kernel<0, 0>;
+    if (policy == 1) return warp_append_kernel<1, 0>;
+    return warp_append_kernel<2, 0>;
+  }
+  if (policy == 0) return warp_append_kernel<0, 1>;
+  if (policy == 1) return warp_append_kernel<1, 1>;
+  return warp_append_kernel<2, 1>;
+}
+
+int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream) {
+  WarpArgs a;
+  a.hp = hp;
+  a.qkv = p.qkv;
+  a.row_stride = p.qkv_row_stride;
+  a.T = p.T;
+  a.B = p.B;
+  a.H = p.Hq + 2 * p.Hkv;
+  a.quads = (a.H + 3) / 4;
+  const int64_t n_head = static_cast<int64_t>(p.T) * a.quads;
+  if (n_head + p.B >= (int64_t{1} << 31)) return FQR_ENOTSUP;
+  a.n_head = static_cast<int>(n_head);
+  a.qw = p.q_norm_w;
+  a.kw = p.k_norm_w;
+  a.cs = p.cos_sin_cache;
+  a.cs_rows = p.cos_sin_rows;
+  a.positions = p.positions;
+  a.q_indptr = p.q_indptr;
+  a.seq_lens = p.seq_lens;
+  a.page_table = p.page_table;
+  a.max_pages = p.max_pages;
+  a.flags = p.flags;
+  const size_t smem = static_cast<size_t>(2 * kHeadDim + 2 * p.B + 1) * sizeof(int);
+  WarpKernel k = select_warp(p.quant_policy, p.rope_style);
+  return launch_persistent(reinterpret_cast<const void*>(k), n_head + p.B, smem, stream,
+                           [&](int grid) { return launch_pdl(k, grid, kThreads, smem, stream, a); });
+}
+
+}  // namespace fqr

@@ -1,0 +1,255 @@
+// fqr_head.cuh -- the per-head arithmetic of the fused append, shared by both
+// schedules (fqr_append_warp.cu, fqr_append_pipe.cu).
+//
+// One 8-lane group owns one 128-element head.  Lane l holds elements
+// [8l, 8l+8) (chunk A) and [64+8l, 64+8l+8) (chunk B) as eight float2 pairs:
+//   y[j]   = elements (8l+2j, 8l+2j+1)        j = 0..3
+//   y[4+j] = elements (64+8l+2j, 64+8l+2j+1)  j = 0..3
+// so a NeoX pair (i, i+64) sits in the same lane (y[j].x <-> y[4+j].x) and a
+// GPT-J pair (2i, 2i+1) in the same float2.  All arithmetic is fp32 with every
+// product and sum rounded on its own (sm_100 f32x2 instructions do two lanes
+// of that at once); the reduction is an xor shuffle inside the group.
+#pragma once
+
+#include "fqr_device.cuh"
+
+namespace fqr {
+
+// Parameters the head arithmetic needs (a sub-struct of each schedule's args).
+struct HeadParams {
+  int Hq, Hkv, page_size, row_bytes, rot;
+  int has_qw, has_kw;
+  float eps, upper_max;
+  char* k_cache;
+  char* v_cache;
+  int64_t k_page_bytes, v_page_bytes;
+  const float* q_scale_inv;
+  const float* k_scale;
+  const float* v_scale;
+  void* out_q;
+  float* q_scale;
+};
+
+// Where one packed row goes.
+struct RowCtx {
+  int t;        // packed row
+  int p_slot;   // sequence position (KV slot)
+  int pos;      // RoPE position
+  int page;     // page id of p_slot (valid when the row has K/V heads to store)
+  int is_last;  // the row is its request's last: its K/V heads also zero the tail
+};
+
+// Shared-memory layout of the fp32 norm weights, 128 per tensor: element e of
+// lane l's slice is stored so that lane l reads its 16 values as four float4
+// at 16-byte lane stride (conflict-free).
+__device__ __forceinline__ int weight_slot(int e) {
+  const int half = e >> 6, r = e & 63, l = r >> 3, k = r & 7;
+  return half * 64 + (k >> 2) * 32 + 4 * l + (k & 3);
+}
+
+// Stage both weight vectors (fp32, permuted) in s_w[0, 256); NULL -> ones.
+__device__ __forceinline__ void stage_weights(float* s_w, const uint16_t* qw, const uint16_t* kw) {
+  for (int i = threadIdx.x; i < 2 * kHeadDim; i += blockDim.x) {
+    const int e = i & (kHeadDim - 1);
+    const uint16_t* w = i < kHeadDim ? qw : kw;
+    const float v = w != nullptr ? __uint_as_float(static_cast<uint32_t>(w[e]) << 16) : 1.0f;
+    s_w[(i & kHeadDim) + weight_slot(e)] = v;
+  }
+}
+
+__device__ __forceinline__ void unpack_pairs(uint4 xa, uint4 xb, float2* y) {
+  y[0] = make_float2(bf16_lo(xa.x), bf16_hi(xa.x));
+  y[1] = make_float2(bf16_lo(xa.y), bf16_hi(xa.y));
+  y[2] = make_float2(bf16_lo(xa.z), bf16_hi(xa.z));
+  y[3] = make_float2(bf16_lo(xa.w), bf16_hi(xa.w));
+  y[4] = make_float2(bf16_lo(xb.x), bf16_hi(xb.x));
+  y[5] = make_float2(bf16_lo(xb.y), bf16_hi(xb.y));
+  y[6] = make_float2(bf16_lo(xb.z), bf16_hi(xb.z));
+  y[7] = make_float2(bf16_lo(xb.w), bf16_hi(xb.w));
+}
+
+__device__ __forceinline__ uint4 pack_bf16_pairs(const float2* y) {
+  return make_uint4(pack_bf16x2(y[0].x, y[0].y), pack_bf16x2(y[1].x, y[1].y),
+                    pack_bf16x2(y[2].x, y[2].y), pack_bf16x2(y[3].x, y[3].y));
+}
+__device__ __forceinline__ uint2 pack_e4m3_pairs(const float2* y) {
+  return make_uint2(pack_e4m3x2(y[0].x, y[0].y) | (pack_e4m3x2(y[1].x, y[1].y) << 16),
+                    pack_e4m3x2(y[2].x, y[2].y) | (pack_e4m3x2(y[3].x, y[3].y) << 16));
+}
+
+__device__ __forceinline__ void divide_pairs(float2* y, float d) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) y[j] = make_float2(__fdiv_rn(y[j].x, d), __fdiv_rn(y[j].y, d));
+}
+
+// Store a head (16 values per lane) into a KV slot / out_q row at `dst`
+// (the head's first byte): bf16 for policy 0, e4m3 otherwise.
+template <int POLICY>
+__device__ __forceinline__ void store_head(char* dst, const float2* y, int l8) {
+  if (POLICY == 0) {
+    st_v4(dst + 16 * l8, pack_bf16_pairs(y));
+    st_v4(dst + 128 + 16 * l8, pack_bf16_pairs(y + 4));
+  } else {
+    st_v2(dst + 8 * l8, pack_e4m3_pairs(y));
+    st_v2(dst + 64 + 8 * l8, pack_e4m3_pairs(y + 4));
+  }
+}
+
+// Zero this head's column of the tail rows [row0 + 1, P) of a page: every
+// tail row is zeroed across its Hkv heads by the Hkv groups together.
+template <int ES>
+__device__ __forceinline__ void zero_tail_column(char* page_base, int row0, int P, int row_bytes,
+                                                 int kh, int l8) {
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  char* col = page_base + static_cast<int64_t>(kh) * kHeadDim * ES + 16 * l8;
+  for (int row = row0 + 1; row < P; ++row) {
+    char* p = col + static_cast<int64_t>(row) * row_bytes;
+    st_v4(p, z);
+    if (ES == 2) st_v4(p + 128, z);
+  }
+}
+
+// Norm + RoPE + quantisation + store of head h of row r.  xa/xb: the lane's two
+// 16-byte slices of the packed head; cs_row: the row's fp32 [cos | sin]
+// (shared or global memory); s_w: staged weights.  gmask: the 8-lane group.
+template <int POLICY, int STYLE>
+__device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& r, int h,
+                                             uint4 xa, uint4 xb, const float* cs_row,
+                                             const float* s_w, int l8, unsigned gmask) {
+  constexpr int ES = POLICY == 0 ? 2 : 1;
+  const int P = a.page_size;
+  float2 y[8];
+  unpack_pairs(xa, xb, y);
+
+  if (h >= a.Hq + a.Hkv) {  // ------------------------------------------ V
+    const int kh = h - a.Hq - a.Hkv;
+    char* page_base = a.v_cache + static_cast<int64_t>(r.page) * a.v_page_bytes;
+    char* dst = page_base + static_cast<int64_t>(r.p_slot % P) * a.row_bytes + kh * kHeadDim * ES;
+    if (POLICY == 0) {  // bit copy
+      st_v4(dst + 16 * l8, xa);
+      st_v4(dst + 128 + 16 * l8, xb);
+    } else {
+      divide_pairs(y, __ldg(a.v_scale));
+      store_head<POLICY>(dst, y, l8);
+    }
+    if (r.is_last) zero_tail_column<ES>(page_base, r.p_slot % P, P, a.row_bytes, kh, l8);
+    return;
+  }
+
+  const bool is_q = h < a.Hq;
+  // ------------------------------------------------------------ cos / sin
+  float2 c[4], s[4];
+  if (STYLE == 0) {  // NeoX, rot == 128: pair k of chunk A is (8l+k, 64+8l+k)
+    const float4 c0 = *reinterpret_cast<const float4*>(cs_row + 8 * l8);
+    const float4 c1 = *reinterpret_cast<const float4*>(cs_row + 8 * l8 + 4);
+    const float4 s0 = *reinterpret_cast<const float4*>(cs_row + 64 + 8 * l8);
+    const float4 s1 = *reinterpret_cast<const float4*>(cs_row + 68 + 8 * l8);
+    c[0] = make_float2(c0.x, c0.y); c[1] = make_float2(c0.z, c0.w);
+    c[2] = make_float2(c1.x, c1.y); c[3] = make_float2(c1.z, c1.w);
+    s[0] = make_float2(s0.x, s0.y); s[1] = make_float2(s0.z, s0.w);
+    s[2] = make_float2(s1.x, s1.y); s[3] = make_float2(s1.z, s1.w);
+  } else {  // GPT-J: y[j] is pair i = 4l + j (chunk A), y[4+j] pair 32 + 4l + j
+    const int half = a.rot >> 1;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int ia = 4 * l8 + j, ib = 32 + 4 * l8 + j;
+      c[j].x = ia < half ? cs_row[ia] : 0.0f;
+      s[j].x = ia < half ? cs_row[half + ia] : 0.0f;
+      c[j].y = ib < half ? cs_row[ib] : 0.0f;
+      s[j].y = ib < half ? cs_row[half + ib] : 0.0f;
+    }
+  }
+
+  // -------------------------------------------------------------- RMSNorm
+  if (is_q ? a.has_qw : a.has_kw) {
+    float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc = fma2(y[j], y[j], acc);
+    float ss = acc.x + acc.y;
+    ss += __shfl_xor_sync(gmask, ss, 4);
+    ss += __shfl_xor_sync(gmask, ss, 2);
+    ss += __shfl_xor_sync(gmask, ss, 1);
+    const float inv = __frcp_rn(__fsqrt_rn(__fadd_rn(ss * (1.0f / kHeadDim), a.eps)));
+    const float2 iv = make_float2(inv, inv);
+    const float* wv = s_w + (is_q ? 0 : kHeadDim) + 4 * l8;
+    const float4 w0 = *reinterpret_cast<const float4*>(wv);
+    const float4 w1 = *reinterpret_cast<const float4*>(wv + 32);
+    const float4 w2 = *reinterpret_cast<const float4*>(wv + 64);
+    const float4 w3 = *reinterpret_cast<const float4*>(wv + 96);
+    const float2 w[8] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w),
+                         make_float2(w1.x, w1.y), make_float2(w1.z, w1.w),
+                         make_float2(w2.x, w2.y), make_float2(w2.z, w2.w),
+                         make_float2(w3.x, w3.y), make_float2(w3.z, w3.w)};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = mul2(mul2(y[j], iv), w[j]);
+  }
+
+  // ----------------------------------------------------------------- RoPE
+  if (STYLE == 0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 ac = mul2(y[j], c[j]), bs = mul2(y[4 + j], s[j]);
+      const float2 bc = mul2(y[4 + j], c[j]), as = mul2(y[j], s[j]);
+      y[j] = add2(ac, make_float2(-bs.x, -bs.y));
+      y[4 + j] = add2(bc, as);
+    }
+  } else {  // dims >= rot_dim pass through untouched
+    const int half = a.rot >> 1;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (4 * l8 + j < half) rotate_pair(y[j].x, y[j].y, c[j].x, s[j].x);
+      if (32 + 4 * l8 + j < half) rotate_pair(y[4 + j].x, y[4 + j].y, c[j].y, s[j].y);
+    }
+  }
+
+  // --------------------------------------------------------------- output
+  if (is_q) {
+    char* dst = static_cast<char*>(a.out_q) +
+                (static_cast<int64_t>(r.t) * a.Hq + h) * kHeadDim * ES;
+    if (POLICY == 1) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fmaxf(fabsf(y[j].x), fabsf(y[j].y)));
+      amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 4));
+      amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 2));
+      amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 1));
+      const float qs = __fdiv_rn(fmaxf(amax, 1e-6f), a.upper_max);
+      if (l8 == 0) a.q_scale[static_cast<int64_t>(r.t) * a.Hq + h] = qs;
+      divide_pairs(y, qs);
+    } else if (POLICY == 2) {
+      const float qsi = __ldg(a.q_scale_inv);
+      const float2 qv = make_float2(qsi, qsi);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[j] = mul2(y[j], qv);
+    }
+    store_head<POLICY>(dst, y, l8);
+  } else {  // ------------------------------------------------------------ K
+    const int kh = h - a.Hq;
+    char* page_base = a.k_cache + static_cast<int64_t>(r.page) * a.k_page_bytes;
+    char* dst = page_base + static_cast<int64_t>(r.p_slot % P) * a.row_bytes + kh * kHeadDim * ES;
+    if (POLICY != 0) divide_pairs(y, __ldg(a.k_scale));
+    store_head<POLICY>(dst, y, l8);
+    if (r.is_last) zero_tail_column<ES>(page_base, r.p_slot % P, P, a.row_bytes, kh, l8);
+  }
+}
+
+// Zero the whole tail (rows [last+1, P), all heads) of request b's last page in
+// both caches: used for requests that append no token in this call.
+template <int ES>
+__device__ __forceinline__ void zero_request_tail(const HeadParams& a, const int32_t* page_table,
+                                                  int max_pages, int b, int L, int lane) {
+  const int P = a.page_size;
+  const int last = (L - 1) % P;
+  const int64_t page = __ldg(page_table + static_cast<int64_t>(b) * max_pages + (L - 1) / P);
+  const int64_t beg = static_cast<int64_t>(last + 1) * a.row_bytes;
+  const int64_t end = static_cast<int64_t>(P) * a.row_bytes;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  char* kb = a.k_cache + page * a.k_page_bytes;
+  char* vb = a.v_cache + page * a.v_page_bytes;
+  for (int64_t off = beg + 16 * lane; off < end; off += 512) {
+    st_v4(kb + off, z);
+    st_v4(vb + off, z);
+  }
+}
+
+}  // namespace fqr

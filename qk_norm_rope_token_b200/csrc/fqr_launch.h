@@ -10,8 +10,34 @@
 
 namespace fqr {
 
+struct HeadParams;
 int launch_append(const fqr_append_params& p, cudaStream_t stream);
+int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream);
+int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream);
 int launch_mla(const fqr_mla_params& p, cudaStream_t stream);
+
+// Launch `kernel(args)` on `stream` with programmatic stream serialization,
+// so that it may begin while the preceding kernel in the stream finishes; the
+// kernel itself waits (griddepcontrol.wait) before reading any input.
+template <class Args>
+int launch_pdl(void (*kernel)(const Args), int grid, int threads, size_t smem,
+               cudaStream_t stream, const Args& args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, args) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return FQR_ECUDA;
+  }
+  return cudaGetLastError() == cudaSuccess ? FQR_OK : FQR_ECUDA;
+}
 
 // Launch a persistent warp-task kernel: one block of kThreads per kWarps
 // tasks, capped at the number of blocks that can be resident on the device at
@@ -34,8 +60,7 @@ int launch_persistent(const void* func, int64_t warp_tasks, size_t smem,
   int64_t need = (warp_tasks + kWarps - 1) / kWarps;
   if (need < 1) need = 1;
   const int64_t cap = static_cast<int64_t>(per_sm) * sms;
-  launch(static_cast<int>(need < cap ? need : cap));
-  return cudaGetLastError() == cudaSuccess ? FQR_OK : FQR_ECUDA;
+  return launch(static_cast<int>(need < cap ? need : cap));
 }
 
 }  // namespace fqr

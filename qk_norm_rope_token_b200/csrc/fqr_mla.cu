@@ -86,6 +86,8 @@ __global__ void __launch_bounds__(kThreads) mla_kernel(const MlaArgs a) {
   const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
 
+  grid_dependency_wait();
+  grid_launch_dependents();
   const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
                static_cast<int64_t>(a.max_blocks) * a.block_size, a.cs_rows};
   if (stage_and_validate(m, s_indptr, s_seq)) return;
@@ -175,7 +177,7 @@ int launch_mla(const fqr_mla_params& p, cudaStream_t stream) {
   const int64_t tasks = static_cast<int64_t>(p.T) * (1 + a.qgroups);
   const size_t smem = static_cast<size_t>(2 * p.B + 1) * sizeof(int);
   return launch_persistent(reinterpret_cast<const void*>(k), tasks, smem, stream,
-                           [&](int grid) { k<<<grid, kThreads, smem, stream>>>(a); });
+                           [&](int grid) { return launch_pdl(k, grid, kThreads, smem, stream, a); });
 }
 
 }  // namespace fqr

@@ -123,8 +123,9 @@ class AppendRun:
     """Device state of one fqr_append_paged call plus what the oracle needs."""
 
     def __init__(self, w, *, fill_seed=11, q_indptr=None, seq_lens=None, page_stride_pad=0,
-                 out_pad=True):
+                 schedule=0):
         self.w = w
+        self.schedule = schedule
         self.q_indptr = np.asarray(w.q_indptr if q_indptr is None else q_indptr, np.int32)
         self.seq_lens = np.asarray(w.seq_lens if seq_lens is None else seq_lens, np.int32)
         es = w.kv_esize
@@ -167,7 +168,7 @@ class AppendRun:
                     q_scale_inv=self.scales["q_scale_inv"] if w.quant_policy == 2 else None,
                     k_scale=self.scales["k_scale"] if w.quant_policy else None,
                     v_scale=self.scales["v_scale"] if w.quant_policy else None,
-                    upper_max=w.upper_max)
+                    upper_max=w.upper_max, schedule=self.schedule)
 
     def launch(self, stream=None):
         fqr.append_paged(self.qkv, self.cs, self.indptr_d, self.seq_d, self.pt_d, self.k_cache,

@@ -92,6 +92,8 @@ APPEND_BAD = {
     "page_size_negative": dict(page_size=-4),
     "tail_rows_overflow": dict(B=16384, page_size=65537),
     "policy_3": dict(quant_policy=3),
+    "schedule_3": dict(schedule=3),
+    "schedule_negative": dict(schedule=-1),
     "rope_style_2": dict(rope_style=2),
     "rot_odd": dict(rope_style=1, rot_dim=63),
     "rot_too_big": dict(rope_style=1, rot_dim=130),

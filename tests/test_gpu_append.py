@@ -21,6 +21,9 @@ if torch.cuda.is_available():
     from tests.gpu_harness import AppendRun, _np
 
 
+SCHEDULES = [1, 2]   # latency, streaming: every case runs under both
+
+
 def run_and_check(w, **kw):
     check_kw = {k: kw.pop(k) for k in list(kw) if k in ("exact_frac_min",)}
     r = AppendRun(w, **kw)
@@ -29,17 +32,19 @@ def run_and_check(w, **kw):
     return r, rep
 
 
+@pytest.mark.parametrize("schedule", [0] + SCHEDULES)
 @pytest.mark.parametrize("name", sorted(workloads.APPEND_CONFIGS))
-def test_named_workload_parity(name):
+def test_named_workload_parity(name, schedule):
     w = workloads.APPEND_CONFIGS[name]()
-    _, rep = run_and_check(w)
-    print(name, rep)
+    _, rep = run_and_check(w, schedule=schedule)
+    print(name, schedule, rep)
     assert not rep.get("flagged")
 
 
-def test_ragged_prefill_malformed_indptr_writes_nothing():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_ragged_prefill_malformed_indptr_writes_nothing(schedule):
     w = workloads.ragged_prefill_fp8()
-    r = AppendRun(w, q_indptr=workloads.malformed_indptr(w))
+    r = AppendRun(w, q_indptr=workloads.malformed_indptr(w), schedule=schedule)
     r.launch()
     rep = r.check()
     assert rep == {"flagged": True}
@@ -62,9 +67,10 @@ SWEEP = [
 ]
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("P,Hq,Hkv,policy,style,rot,norm,pos,pad", SWEEP)
 @pytest.mark.parametrize("seed", [1, 2])
-def test_small_ragged_sweep(P, Hq, Hkv, policy, style, rot, norm, pos, pad, seed):
+def test_small_ragged_sweep(P, Hq, Hkv, policy, style, rot, norm, pos, pad, seed, schedule):
     rng = np.random.default_rng(seed * 1000 + P + Hq)
     B = 7
     n = rng.integers(0, 40, B)
@@ -82,17 +88,18 @@ def test_small_ragged_sweep(P, Hq, Hkv, policy, style, rot, norm, pos, pad, seed
                               rope_style=style, cos_sin_rows=rows, row_pad=pad,
                               positions=positions, q_scale_inv=1 / 0.05, k_scale=0.05,
                               v_scale=0.05)
-    _, rep = run_and_check(w, exact_frac_min=0.95)
+    _, rep = run_and_check(w, exact_frac_min=0.95, schedule=schedule)
     if not norm:
         # without the norm both sides evaluate identical fp32 expressions
         assert rep["q_exact_frac"] == 1.0 and rep.get("k_exact_frac", 1.0) == 1.0
 
 
-def test_requests_without_tokens_only_tails_and_flags():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_requests_without_tokens_only_tails_and_flags(schedule):
     w = workloads.make_append(seed=3, n_new=[0, 0, 0, 0], seq_lens=[0, 5, 16, 33], Hq=8, Hkv=2,
                               page_size=16, max_pages=3, quant_policy=1, cos_sin_rows=40,
                               k_scale=0.05, v_scale=0.05)
-    r, _ = run_and_check(w)
+    r, _ = run_and_check(w, schedule=schedule)
     assert (r.flags.cpu().numpy() == 0).all()
 
 
@@ -108,46 +115,51 @@ BAD = {
 }
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("case", sorted(BAD))
 @pytest.mark.parametrize("policy", [0, 1, 2])
-def test_each_malformed_predicate_writes_nothing(case, policy):
+def test_each_malformed_predicate_writes_nothing(case, policy, schedule):
     w = workloads.make_append(seed=4, n_new=[2, 0, 3], seq_lens=[5, 4, 3], Hq=4, Hkv=2,
                               page_size=4, max_pages=3, quant_policy=policy, cos_sin_rows=11,
                               k_scale=0.05, v_scale=0.05, q_scale_inv=20.0)
     over = {k: np.array(v, np.int32) for k, v in BAD[case].items()}
-    r = AppendRun(w, **over)
+    r = AppendRun(w, schedule=schedule, **over)
     r.launch()
     assert r.check() == {"flagged": True}
     assert (r.flags.cpu().numpy() == -1).all()
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("bad", [-1, 11])
-def test_explicit_position_out_of_range_writes_nothing(bad):
+def test_explicit_position_out_of_range_writes_nothing(bad, schedule):
     w = workloads.make_append(seed=5, n_new=[2, 3], seq_lens=[2, 3], Hq=4, Hkv=2, page_size=4,
                               max_pages=2, cos_sin_rows=11, positions=[0, 1, 2, bad, 4])
-    r = AppendRun(w)
+    r = AppendRun(w, schedule=schedule)
     r.launch()
     assert r.check() == {"flagged": True}
 
 
-def test_largest_batch():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_largest_batch(schedule):
     B = 16384
     rng = np.random.default_rng(8)
     L = rng.integers(1, 64, B)
     w = workloads.make_append(seed=8, n_new=[1] * B, seq_lens=L, Hq=2, Hkv=1, page_size=16,
                               max_pages=4, quant_policy=1, cos_sin_rows=64, k_scale=0.05,
                               v_scale=0.05)
-    run_and_check(w)
+    run_and_check(w, schedule=schedule)
 
 
-def test_padded_page_stride():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_padded_page_stride(schedule):
     w = workloads.make_append(seed=9, n_new=[5, 17, 0, 1], seq_lens=[9, 30, 7, 1], Hq=8,
                               Hkv=2, page_size=16, max_pages=3, quant_policy=2,
                               q_scale_inv=20.0, k_scale=0.05, v_scale=0.05)
-    run_and_check(w, page_stride_pad=256)
+    run_and_check(w, page_stride_pad=256, schedule=schedule)
 
 
-def test_every_bf16_input_through_the_fp8_encoder():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_every_bf16_input_through_the_fp8_encoder(schedule):
     """All 65536 BF16 codes (inf and NaN included) as Q inputs with no norm and
     an identity rotation (GPT-J, rot_dim 2, position 0), static scale 1: the
     payload is the E4M3 encoding of the input itself, and the GPU's packed
@@ -165,7 +177,7 @@ def test_every_bf16_input_through_the_fp8_encoder():
     q[:, :, 2:] = codes.reshape(T, Hq, per_head)
     q[:, :, :2] = 0x3F80                      # the rotated pair stays finite
     w.qkv[:, : Hq * D] = q.reshape(T, Hq * D)
-    r, rep = run_and_check(w)
+    r, rep = run_and_check(w, schedule=schedule)
     assert rep["q_exact_frac"] == 1.0
     # the payload is the encoding of the input value itself (NaN codes equal)
     got = _np(r.out_q).reshape(T, Hq, D)[:, :, 2:].reshape(-1)[:65536]
@@ -173,19 +185,21 @@ def test_every_bf16_input_through_the_fp8_encoder():
     assert (ulp_e4m3(got, want) == 0).all()
 
 
-def test_heads_far_apart_in_scale_normalise_independently():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_heads_far_apart_in_scale_normalise_independently(schedule):
     w = workloads.make_append(seed=12, n_new=[3, 2], seq_lens=[40, 2], Hq=16, Hkv=4,
                               page_size=16, max_pages=3, quant_policy=0)
     x = bf16_bits_to_f32(w.qkv).copy()
     for h in range(0, 24, 2):
         x[:, h * D:(h + 1) * D] *= 1e3
     w.qkv = (x.view(np.uint32) >> 16).astype(np.uint16)
-    run_and_check(w)
+    run_and_check(w, schedule=schedule)
 
 
-def test_non_default_stream():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_non_default_stream(schedule):
     w = workloads.tiny_decode_bf16()
-    r = AppendRun(w)
+    r = AppendRun(w, schedule=schedule)
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
         r.launch(stream=s)
@@ -193,9 +207,10 @@ def test_non_default_stream():
     r.check()
 
 
-def test_cuda_graph_capture_and_replay_is_bitwise_eager():
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_cuda_graph_capture_and_replay_is_bitwise_eager(schedule):
     w = workloads.fp8_decode_dynamic()
-    r = AppendRun(w)
+    r = AppendRun(w, schedule=schedule)
     r.launch()
     torch.cuda.synchronize()
     eager = (r.out_q.clone(), r.q_scale.clone(), r.k_store.clone(), r.v_store.clone(),
