@@ -70,6 +70,9 @@ def parse_args(argv=None):
                     help="profiling run: only --workload (or mla_decode), --steps eager launches, "
                          "no graphs, no e2e / per-config / CPU legs, no JSON line")
     ap.add_argument("--mla", action="store_true", help="with --profile: the MLA workload")
+    ap.add_argument("--small-cache", action="store_true",
+                    help="with --profile: wrap sequence lengths to 1024 (same bytes per call, "
+                         "a cache of 1024 slots per request)")
     return ap.parse_args(argv)
 
 
@@ -187,17 +190,21 @@ class AppendBench:
     """R replicas of one append workload sharing one pair of KV caches."""
 
     def __init__(self, name, torch, fqr, device, min_bytes=3 * L2_BYTES, max_replicas=64,
-                 seed_offset=0, schedule=0):
+                 seed_offset=0, schedule=0, small_cache=False):
         self.torch, self.fqr, self.dev = torch, fqr, device
         self.schedule = schedule
-        base = workloads.APPEND_CONFIGS[name]()
+        make = workloads.APPEND_CONFIGS[name]
+        if small_cache:
+            def make(seed=None, _f=workloads.APPEND_CONFIGS[name]):
+                return workloads.shrink_cache(_f() if seed is None else _f(seed=seed))
+        base = make()
         self.name = base.name
         per = workloads.append_bytes(base)["total"]
         self.R = int(min(max_replicas, max(2, math.ceil(min_bytes / per))))
         ws = []
         for r in range(self.R):
             sd = base.seed + seed_offset + 7919 * r
-            ws.append(base if sd == base.seed else workloads.APPEND_CONFIGS[name](seed=sd))
+            ws.append(base if sd == base.seed else make(seed=sd))
         self.ws = ws
         self.bytes = [workloads.append_bytes(w)["total"] for w in ws]
         self.T = base.T
@@ -590,7 +597,7 @@ def run_profile(args, torch, fqr, dev):
         b = MlaBench(torch, fqr, dev, max_replicas=args.replicas or 2)
     else:
         b = AppendBench(args.workload, torch, fqr, dev, max_replicas=args.replicas or 2,
-                        schedule=args.schedule)
+                        schedule=args.schedule, small_cache=args.small_cache)
     h = torch.cuda.current_stream().cuda_stream
     for i in range(args.warmup + args.steps):
         b.launch(i, h)

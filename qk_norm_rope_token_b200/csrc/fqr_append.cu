@@ -19,6 +19,7 @@ constexpr int kStreamRowsPerSm = 4;
 int launch_append(const fqr_append_params& p, cudaStream_t stream) {
   HeadParams hp;
   const int es = p.quant_policy == 0 ? 2 : 1;
+  hp.pdiv = FastDiv(static_cast<uint32_t>(p.page_size));
   hp.Hq = p.Hq;
   hp.Hkv = p.Hkv;
   hp.page_size = p.page_size;

@@ -35,11 +35,12 @@ constexpr int kFixedSmem = 1280;  // barriers (128) + fp32 weights (1024) + spar
 
 // Stage header, written by the producer before it arrives on "full".
 struct StageInfo {
-  int p_slot, page, pos, is_last;
+  int slot_row, page, pos, is_last;
 };
 
 struct PipeArgs {
   HeadParams hp;
+  FastDiv cdiv;  // division by nchunks
   const uint16_t* qkv;
   int64_t row_stride;
   int T, B, H;
@@ -76,8 +77,8 @@ __device__ void report_timeout(const PipeArgs& a) {
 // Unit u: packed row t, heads [h0, h0 + nh).
 __device__ __forceinline__ void unit_heads(const PipeArgs& a, int64_t u, int& t, int& h0,
                                            int& nh) {
-  t = static_cast<int>(u / a.nchunks);
-  h0 = static_cast<int>(u - static_cast<int64_t>(t) * a.nchunks) * a.chunk_heads;
+  t = static_cast<int>(a.cdiv.div(static_cast<uint32_t>(u)));
+  h0 = (static_cast<int>(u) - t * a.nchunks) * a.chunk_heads;
   nh = min(a.H - h0, a.chunk_heads);
 }
 
@@ -101,9 +102,11 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
   const int S = a.stages;
   int ok = 1;
   int issued = pre;  // stages whose head copies are in flight or consumed
+  int s = 0;         // stage of unit i
+  uint32_t eph = 1;  // parity of the empty-phase to wait for (previous use of stage s)
   for (int i0 = 0; i0 < nunits && ok; i0 += 32) {
     // lane j prepares unit i0 + j in parallel with the others
-    StageInfo info{0, 0, 0, 0};  // p_slot, page, pos, is_last
+    StageInfo info{0, 0, 0, 0};  // slot_row, page, pos, is_last
     int need_cs = 0;
     if (i0 + lane < nunits) {
       int t, h0, nh;
@@ -111,12 +114,12 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
       const int b = request_of_row(s_indptr, a.B, t);
       const int end = s_indptr[b + 1];
       const int p = t + s_seq[b] - end;
-      info.p_slot = p;
+      const int pidx = static_cast<int>(a.hp.pdiv.div(static_cast<uint32_t>(p)));
+      info.slot_row = p - pidx * a.hp.page_size;
       info.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : p;
       info.is_last = t == end - 1;
       if (h0 + nh > a.hp.Hq)  // the unit holds K or V heads: it needs the page id
-        info.page =
-            __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + p / a.hp.page_size);
+        info.page = __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx);
       need_cs = (h0 < a.hp.Hq + a.hp.Hkv) && a.cs_bulk;
     }
     const int n = min(32, nunits - i0);
@@ -124,11 +127,11 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
       // position first: the cos/sin copy must not wait for the page-id load
       const int posj = __shfl_sync(0xffffffffu, info.pos, j);
       const int csj = __shfl_sync(0xffffffffu, need_cs, j);
-      const int i = i0 + j, s = i % S;
+      const int i = i0 + j;
       uint64_t* fb = &full[s];
       unsigned char* st = stages + static_cast<size_t>(s) * a.stage_bytes;
       if (lane == 0) {
-        if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1)) ok = 0;
+        if (i >= S && !mbar_wait(&empty[s], eph)) ok = 0;
         if (ok) {
           fence_proxy_async_smem();
           if (i >= pre) {
@@ -144,12 +147,16 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      const StageInfo sj{__shfl_sync(0xffffffffu, info.p_slot, j),
+      const StageInfo sj{__shfl_sync(0xffffffffu, info.slot_row, j),
                          __shfl_sync(0xffffffffu, info.page, j), posj,
                          __shfl_sync(0xffffffffu, info.is_last, j)};
       if (lane == 0) {
         *reinterpret_cast<StageInfo*>(st) = sj;
         mbar_arrive(fb);  // release: the header is visible once the phase completes
+      }
+      if (++s == S) {
+        s = 0;
+        eph ^= 1u;
       }
     }
   }
@@ -163,7 +170,7 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
 }
 
 // ------------------------------------------------------------ consumers --
-template <int POLICY, int STYLE>
+template <int POLICY, int STYLE, bool CSB>
 __device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t* full,
                         uint64_t* empty, const float* s_w, int64_t u0, int nunits) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -174,17 +181,18 @@ __device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t
   int t = static_cast<int>(u0 / a.nchunks);
   int c = static_cast<int>(u0 - static_cast<int64_t>(t) * a.nchunks);
   int rot = 0;  // quad -> warp rotation, advanced by nq every unit
+  int s = 0;
+  uint32_t ph = 0;
   for (int i = 0; i < nunits; ++i) {
-    const int s = i % S;
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / S) & 1))) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph))) {
       report_timeout(a);
       return;
     }
     const unsigned char* st = stages + static_cast<size_t>(s) * a.stage_bytes;
     const StageInfo info = *reinterpret_cast<const StageInfo*>(st);
-    const RowCtx r{t, info.p_slot, info.pos, info.page, info.is_last};
-    const float* cs_row = a.cs_bulk ? reinterpret_cast<const float*>(st + 16)
-                                    : a.cs + static_cast<int64_t>(info.pos) * a.hp.rot;
+    const RowCtx r{t, info.slot_row, info.pos, info.page, info.is_last};
+    const float* cs_row = CSB ? reinterpret_cast<const float*>(st + 16)
+                              : a.cs + static_cast<int64_t>(info.pos) * a.hp.rot;
     const int h0 = c * a.chunk_heads, nh = min(a.H - h0, a.chunk_heads);
     const int nq = (nh + 3) >> 2;
     int q = warp - rot;
@@ -193,12 +201,20 @@ __device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t
       const int hl = 4 * q + g;
       if (hl < nh) {
         const unsigned char* src = st + 16 + a.cs_bytes + hl * (kHeadDim * 2) + 16 * l8;
-        process_head<POLICY, STYLE>(a.hp, r, h0 + hl, ld_smem_v4(src), ld_smem_v4(src + 128),
-                                    cs_row, s_w, l8, gmask);
+        if (CSB)
+          process_head<POLICY, STYLE, true>(a.hp, r, h0 + hl, ld_smem_v4(src),
+                                            ld_smem_v4(src + 128), cs_row, s_w, l8, gmask);
+        else
+          process_head<POLICY, STYLE, false>(a.hp, r, h0 + hl, ld_smem_v4(src),
+                                             ld_smem_v4(src + 128), cs_row, s_w, l8, gmask);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == S) {
+      s = 0;
+      ph ^= 1u;
+    }
     rot = (rot + nq) & (kConsumers - 1);
     if (++c == a.nchunks) {
       c = 0;
@@ -221,7 +237,7 @@ __device__ void zero_empty_request_tails(const PipeArgs& a, const int* s_indptr,
 }
 
 template <int POLICY, int STYLE>
-__global__ void __launch_bounds__(kPipeThreads) pipe_append_kernel(const PipeArgs a) {
+__global__ void __launch_bounds__(kPipeThreads, 2) pipe_append_kernel(const PipeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kMaxStages;
@@ -276,7 +292,14 @@ __global__ void __launch_bounds__(kPipeThreads) pipe_append_kernel(const PipeArg
     produce(a, stages, full, empty, s_indptr, s_seq, u0, nunits, pre);
   } else {
     zero_empty_request_tails<POLICY>(a, s_indptr, s_seq);
-    consume<POLICY, STYLE>(a, stages, full, empty, s_w, u0, nunits);
+    if constexpr (STYLE == 0) {  // NeoX rows are 128 wide: always staged
+      consume<POLICY, STYLE, true>(a, stages, full, empty, s_w, u0, nunits);
+    } else {
+      if (a.cs_bulk)
+        consume<POLICY, STYLE, true>(a, stages, full, empty, s_w, u0, nunits);
+      else
+        consume<POLICY, STYLE, false>(a, stages, full, empty, s_w, u0, nunits);
+    }
   }
 }
 
@@ -333,9 +356,11 @@ int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStr
   a.chunk_heads = hc;
   a.nchunks = (a.H + hc - 1) / hc;
   a.units = static_cast<int64_t>(p.T) * a.nchunks;
+  if (a.units >= (int64_t{1} << 31)) return FQR_ENOTSUP;
+  a.cdiv = FastDiv(static_cast<uint32_t>(a.nchunks));
   a.stage_bytes = stage_bytes(hc);
-  // pipeline depth: aim at two resident blocks per SM, never deeper than the
-  // units a block will see
+  // pipeline depth: aim at two resident blocks per SM (the register budget of
+  // the consumers), never deeper than the units a block will see
   const int64_t per_block_budget = smem_sm / 2 - 1024;
   int S = static_cast<int>((per_block_budget - kFixedSmem - meta) / a.stage_bytes);
   S = S < 1 ? 1 : (S > kMaxStages ? kMaxStages : S);

@@ -20,6 +20,7 @@ namespace fqr {
 
 struct WarpArgs {
   HeadParams hp;
+  FastDiv qdiv;  // division by quads
   const uint16_t* qkv;
   int64_t row_stride;
   int T, B, H, quads, n_head;
@@ -37,7 +38,7 @@ struct WarpArgs {
 
 __device__ __forceinline__ void warp_load_head(const WarpArgs& a, int w, int g, int l8, uint4& xa,
                                                uint4& xb) {
-  const int t = w / a.quads;
+  const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
   const int h = (w - t * a.quads) * 4 + g;
   if (h < a.H) {
     const uint16_t* src = a.qkv + static_cast<int64_t>(t) * a.row_stride + h * kHeadDim + 8 * l8;
@@ -75,21 +76,21 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
     if (w < a.n_head) {
       const uint4 xa = pa, xb = pb;
       if (w + nwarps < a.n_head) warp_load_head(a, w + nwarps, g, l8, pa, pb);
-      const int t = w / a.quads;
+      const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
       const int h = (w - t * a.quads) * 4 + g;
       if (h >= a.H) continue;  // the whole 8-lane group skips together
       const int b = request_of_row(s_indptr, a.B, t);
       const int end = s_indptr[b + 1];
+      const int p_slot = t + s_seq[b] - end;
+      const int pidx = static_cast<int>(a.hp.pdiv.div(static_cast<uint32_t>(p_slot)));
       RowCtx r;
       r.t = t;
-      r.p_slot = t + s_seq[b] - end;
-      r.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : r.p_slot;
+      r.slot_row = p_slot - pidx * a.hp.page_size;
+      r.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : p_slot;
       r.is_last = t == end - 1;
-      r.page = h >= a.hp.Hq
-                   ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + r.p_slot / a.hp.page_size)
-                   : 0;
+      r.page = h >= a.hp.Hq ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx) : 0;
       const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
-      process_head<POLICY, STYLE>(a.hp, r, h, xa, xb, cs_row, s_w, l8, gmask);
+      process_head<POLICY, STYLE, false>(a.hp, r, h, xa, xb, cs_row, s_w, l8, gmask);
     } else {
       const int b = w - a.n_head;  // request task: tail of a request without new rows
       const int L = s_seq[b];
@@ -124,6 +125,7 @@ int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStr
   const int64_t n_head = static_cast<int64_t>(p.T) * a.quads;
   if (n_head + p.B >= (int64_t{1} << 31)) return FQR_ENOTSUP;
   a.n_head = static_cast<int>(n_head);
+  a.qdiv = FastDiv(static_cast<uint32_t>(a.quads));
   a.qw = p.q_norm_w;
   a.kw = p.k_norm_w;
   a.cs = p.cos_sin_cache;

@@ -17,6 +17,7 @@ namespace fqr {
 
 // Parameters the head arithmetic needs (a sub-struct of each schedule's args).
 struct HeadParams {
+  FastDiv pdiv;  // division by page_size
   int Hq, Hkv, page_size, row_bytes, rot;
   int has_qw, has_kw;
   float eps, upper_max;
@@ -32,12 +33,36 @@ struct HeadParams {
 
 // Where one packed row goes.
 struct RowCtx {
-  int t;        // packed row
-  int p_slot;   // sequence position (KV slot)
-  int pos;      // RoPE position
-  int page;     // page id of p_slot (valid when the row has K/V heads to store)
-  int is_last;  // the row is its request's last: its K/V heads also zero the tail
+  int t;         // packed row
+  int slot_row;  // row of the KV slot inside its page (p_slot % page_size)
+  int pos;       // RoPE position
+  int page;      // page id of the KV slot (valid when the row has K/V heads to store)
+  int is_last;   // the row is its request's last: its K/V heads also zero the tail
 };
+
+__device__ __forceinline__ float4 lds_f4(const float* p) {
+  float4 r;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "r"(smem_addr(p)));
+  return r;
+}
+// cos/sin row reads: shared memory when the row was staged there, else the
+// read-only path from global memory.
+template <bool CS_SMEM>
+__device__ __forceinline__ float4 ld_cs4(const float* p) {
+  if (CS_SMEM) return lds_f4(p);
+  return __ldg(reinterpret_cast<const float4*>(p));
+}
+template <bool CS_SMEM>
+__device__ __forceinline__ float ld_cs1(const float* p) {
+  if (CS_SMEM) {
+    float r;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(r) : "r"(smem_addr(p)));
+    return r;
+  }
+  return __ldg(p);
+}
 
 // Shared-memory layout of the fp32 norm weights, 128 per tensor: element e of
 // lane l's slice is stored so that lane l reads its 16 values as four float4
@@ -112,7 +137,7 @@ __device__ __forceinline__ void zero_tail_column(char* page_base, int row0, int 
 // Norm + RoPE + quantisation + store of head h of row r.  xa/xb: the lane's two
 // 16-byte slices of the packed head; cs_row: the row's fp32 [cos | sin]
 // (shared or global memory); s_w: staged weights.  gmask: the 8-lane group.
-template <int POLICY, int STYLE>
+template <int POLICY, int STYLE, bool CS_SMEM>
 __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& r, int h,
                                              uint4 xa, uint4 xb, const float* cs_row,
                                              const float* s_w, int l8, unsigned gmask) {
@@ -124,7 +149,7 @@ __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& 
   if (h >= a.Hq + a.Hkv) {  // ------------------------------------------ V
     const int kh = h - a.Hq - a.Hkv;
     char* page_base = a.v_cache + static_cast<int64_t>(r.page) * a.v_page_bytes;
-    char* dst = page_base + static_cast<int64_t>(r.p_slot % P) * a.row_bytes + kh * kHeadDim * ES;
+    char* dst = page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
     if (POLICY == 0) {  // bit copy
       st_v4(dst + 16 * l8, xa);
       st_v4(dst + 128 + 16 * l8, xb);
@@ -132,7 +157,7 @@ __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& 
       divide_pairs(y, __ldg(a.v_scale));
       store_head<POLICY>(dst, y, l8);
     }
-    if (r.is_last) zero_tail_column<ES>(page_base, r.p_slot % P, P, a.row_bytes, kh, l8);
+    if (r.is_last) zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
     return;
   }
 
@@ -140,10 +165,10 @@ __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& 
   // ------------------------------------------------------------ cos / sin
   float2 c[4], s[4];
   if (STYLE == 0) {  // NeoX, rot == 128: pair k of chunk A is (8l+k, 64+8l+k)
-    const float4 c0 = *reinterpret_cast<const float4*>(cs_row + 8 * l8);
-    const float4 c1 = *reinterpret_cast<const float4*>(cs_row + 8 * l8 + 4);
-    const float4 s0 = *reinterpret_cast<const float4*>(cs_row + 64 + 8 * l8);
-    const float4 s1 = *reinterpret_cast<const float4*>(cs_row + 68 + 8 * l8);
+    const float4 c0 = ld_cs4<CS_SMEM>(cs_row + 8 * l8);
+    const float4 c1 = ld_cs4<CS_SMEM>(cs_row + 8 * l8 + 4);
+    const float4 s0 = ld_cs4<CS_SMEM>(cs_row + 64 + 8 * l8);
+    const float4 s1 = ld_cs4<CS_SMEM>(cs_row + 68 + 8 * l8);
     c[0] = make_float2(c0.x, c0.y); c[1] = make_float2(c0.z, c0.w);
     c[2] = make_float2(c1.x, c1.y); c[3] = make_float2(c1.z, c1.w);
     s[0] = make_float2(s0.x, s0.y); s[1] = make_float2(s0.z, s0.w);
@@ -153,10 +178,10 @@ __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& 
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int ia = 4 * l8 + j, ib = 32 + 4 * l8 + j;
-      c[j].x = ia < half ? cs_row[ia] : 0.0f;
-      s[j].x = ia < half ? cs_row[half + ia] : 0.0f;
-      c[j].y = ib < half ? cs_row[ib] : 0.0f;
-      s[j].y = ib < half ? cs_row[half + ib] : 0.0f;
+      c[j].x = ia < half ? ld_cs1<CS_SMEM>(cs_row + ia) : 0.0f;
+      s[j].x = ia < half ? ld_cs1<CS_SMEM>(cs_row + half + ia) : 0.0f;
+      c[j].y = ib < half ? ld_cs1<CS_SMEM>(cs_row + ib) : 0.0f;
+      s[j].y = ib < half ? ld_cs1<CS_SMEM>(cs_row + half + ib) : 0.0f;
     }
   }
 
@@ -172,10 +197,10 @@ __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& 
     const float inv = __frcp_rn(__fsqrt_rn(__fadd_rn(ss * (1.0f / kHeadDim), a.eps)));
     const float2 iv = make_float2(inv, inv);
     const float* wv = s_w + (is_q ? 0 : kHeadDim) + 4 * l8;
-    const float4 w0 = *reinterpret_cast<const float4*>(wv);
-    const float4 w1 = *reinterpret_cast<const float4*>(wv + 32);
-    const float4 w2 = *reinterpret_cast<const float4*>(wv + 64);
-    const float4 w3 = *reinterpret_cast<const float4*>(wv + 96);
+    const float4 w0 = lds_f4(wv);
+    const float4 w1 = lds_f4(wv + 32);
+    const float4 w2 = lds_f4(wv + 64);
+    const float4 w3 = lds_f4(wv + 96);
     const float2 w[8] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w),
                          make_float2(w1.x, w1.y), make_float2(w1.z, w1.w),
                          make_float2(w2.x, w2.y), make_float2(w2.z, w2.w),
@@ -226,10 +251,10 @@ __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& 
   } else {  // ------------------------------------------------------------ K
     const int kh = h - a.Hq;
     char* page_base = a.k_cache + static_cast<int64_t>(r.page) * a.k_page_bytes;
-    char* dst = page_base + static_cast<int64_t>(r.p_slot % P) * a.row_bytes + kh * kHeadDim * ES;
+    char* dst = page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
     if (POLICY != 0) divide_pairs(y, __ldg(a.k_scale));
     store_head<POLICY>(dst, y, l8);
-    if (r.is_last) zero_tail_column<ES>(page_base, r.p_slot % P, P, a.row_bytes, kh, l8);
+    if (r.is_last) zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
   }
 }
 
@@ -239,8 +264,9 @@ template <int ES>
 __device__ __forceinline__ void zero_request_tail(const HeadParams& a, const int32_t* page_table,
                                                   int max_pages, int b, int L, int lane) {
   const int P = a.page_size;
-  const int last = (L - 1) % P;
-  const int64_t page = __ldg(page_table + static_cast<int64_t>(b) * max_pages + (L - 1) / P);
+  const uint32_t pidx = a.pdiv.div(static_cast<uint32_t>(L - 1));
+  const int last = L - 1 - static_cast<int>(pidx) * P;
+  const int64_t page = __ldg(page_table + static_cast<int64_t>(b) * max_pages + pidx);
   const int64_t beg = static_cast<int64_t>(last + 1) * a.row_bytes;
   const int64_t end = static_cast<int64_t>(P) * a.row_bytes;
   const uint4 z = make_uint4(0u, 0u, 0u, 0u);

@@ -356,3 +356,28 @@ def mla_bytes(w: MlaWorkload) -> dict:
     cache_e = 1 if w.cache_fp8 else 2
     writes = T * w.Hq * w.rope_dim * 2 + T * w.width * cache_e + 4 * B
     return {"read": int(reads), "write": int(writes), "total": int(reads + writes)}
+
+
+def shrink_cache(w: AppendWorkload, max_len: int = 1024) -> AppendWorkload:
+    """A copy of a decode-style workload on a smaller cache, for profiling.
+
+    Post-append lengths wrap modulo max_len (a multiple of the page size), so
+    every request keeps its position inside its last page -- hence the same
+    tail size and the same bytes per call -- while the page table and the
+    cache shrink to max_len / page_size pages per request."""
+    import copy
+    if max_len % w.page_size:
+        raise ValueError("max_len must be a multiple of the page size")
+    n = np.diff(w.q_indptr)
+    L = w.seq_lens.astype(np.int64)
+    L2 = np.where(L > 0, (L - 1) % max_len + 1, 0)
+    if np.any(L2 < n):
+        raise ValueError("a request appends more rows than max_len")
+    s = copy.copy(w)
+    s.seq_lens = L2.astype(np.int32)
+    mp = max_len // w.page_size
+    rng = rng_for(w.seed + 99)
+    s.num_pages = w.B * mp
+    s.page_table = rng.permutation(s.num_pages).astype(np.int32).reshape(w.B, mp)
+    s.cos_sin = w.cos_sin[:max_len].copy()
+    return s
