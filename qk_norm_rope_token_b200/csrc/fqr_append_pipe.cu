@@ -274,11 +274,12 @@ __global__ void __launch_bounds__(kPipeThreads, 2) pipe_append_kernel(const Pipe
     for (int i = 0; i < pre; ++i)
       issue_heads(a, stages + static_cast<size_t>(i) * a.stage_bytes, u0 + i, &full[i]);
   }
-  stage_weights(s_w, a.qw, a.kw);
+  const MetaRegs meta = meta_prefetch(a.q_indptr, a.seq_lens, a.B);
+  weight_store(s_w, weight_prefetch(a.qw, a.kw));
 
   const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
                static_cast<int64_t>(a.max_pages) * a.hp.page_size, a.cs_rows};
-  if (stage_and_validate(m, s_indptr, s_seq)) {
+  if (stage_and_validate(m, s_indptr, s_seq, meta)) {
     if (producer && lane == 0) {  // drain the copies issued before the verdict
       for (int i = 0; i < pre; ++i) {
         mbar_arrive(&full[i]);

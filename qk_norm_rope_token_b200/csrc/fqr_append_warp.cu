@@ -8,6 +8,10 @@
 //     16-byte loads per lane need no metadata and are issued before the
 //     validation prologue; the next task's loads are issued before the current
 //     task is computed.
+//   * the first task also reads its own request's metadata in that first
+//     round trip (request guessed as b = t) and, when it is consistent and
+//     in bounds, issues its page-id and cos/sin loads before the prologue, so
+//     the second dependent round trip overlaps the batch validation.
 //   * every block stages q_indptr / seq_lens in shared memory and validates the
 //     whole batch (stage_and_validate); a malformed batch writes only flags.
 //   * the K/V heads of a request's last new row also zero their column of the
@@ -63,19 +67,63 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   grid_dependency_wait();
   grid_launch_dependents();
 
+  // ---- first round trip: every load that needs no metadata -- the batch
+  // metadata this thread stages, the norm weights, the first task's packed
+  // heads and its own request's metadata (request guessed as b = t: one new
+  // row per request, the decode case).
+  const MetaRegs meta = meta_prefetch(a.q_indptr, a.seq_lens, a.B);
+  const float wreg = weight_prefetch(a.qw, a.kw);
   uint4 pa = make_uint4(0u, 0u, 0u, 0u), pb = pa;
-  if (gwarp < a.n_head) warp_load_head(a, gwarp, g, l8, pa, pb);
-  stage_weights(s_w, a.qw, a.kw);
+  const bool head0 = gwarp < a.n_head;
+  int t0 = 0, h0 = a.H, gb = 0, e_lo = 0, e_hi = 0, e_L = 0;
+  int64_t e_pos = 0;
+  if (head0) {
+    t0 = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(gwarp)));
+    h0 = (gwarp - t0 * a.quads) * 4 + g;
+    warp_load_head(a, gwarp, g, l8, pa, pb);
+    gb = t0 < a.B - 1 ? t0 : a.B - 1;
+    e_lo = __ldg(a.q_indptr + gb);
+    e_hi = __ldg(a.q_indptr + gb + 1);
+    e_L = __ldg(a.seq_lens + gb);
+    if (a.positions != nullptr) e_pos = __ldg(a.positions + t0);
+  }
+  // ---- second round trip, started before the validation prologue when the
+  // row's own metadata is consistent and every address it yields is in
+  // bounds (the prologue still decides whether anything is written).
+  RowCtx r0{t0, 0, 0, 0, 0};
+  float2 c0[4], s0[4];
+  bool early = false;
+  if (head0 && h0 < a.H && e_lo <= t0 && t0 < e_hi) {
+    const int p = t0 + e_L - e_hi;
+    const int64_t pos = a.positions != nullptr ? e_pos : static_cast<int64_t>(p);
+    if (p >= 0 && p < static_cast<int64_t>(a.max_pages) * a.hp.page_size && pos >= 0 &&
+        pos < a.cs_rows) {
+      early = true;
+      const int pidx = static_cast<int>(a.hp.pdiv.div(static_cast<uint32_t>(p)));
+      r0.slot_row = p - pidx * a.hp.page_size;
+      r0.pos = static_cast<int>(pos);
+      r0.is_last = t0 == e_hi - 1;
+      if (h0 >= a.hp.Hq)
+        r0.page = __ldg(a.page_table + static_cast<int64_t>(gb) * a.max_pages + pidx);
+      if (h0 < a.hp.Hq + a.hp.Hkv)
+        load_cs<STYLE, false>(a.cs + pos * a.hp.rot, a.hp.rot, l8, c0, s0);
+    }
+  }
+  weight_store(s_w, wreg);
 
   const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
                static_cast<int64_t>(a.max_pages) * a.hp.page_size, a.cs_rows};
-  if (stage_and_validate(m, s_indptr, s_seq)) return;
+  if (stage_and_validate(m, s_indptr, s_seq, meta)) return;
 
   const int n_tasks = a.n_head + a.B;
   for (int w = gwarp; w < n_tasks; w += nwarps) {
     if (w < a.n_head) {
       const uint4 xa = pa, xb = pb;
       if (w + nwarps < a.n_head) warp_load_head(a, w + nwarps, g, l8, pa, pb);
+      if (w == gwarp && early) {  // the batch is valid: the early lookups stand
+        process_head_cs<POLICY, STYLE>(a.hp, r0, h0, xa, xb, c0, s0, s_w, l8, gmask);
+        continue;
+      }
       const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
       const int h = (w - t * a.quads) * 4 + g;
       if (h >= a.H) continue;  // the whole 8-lane group skips together

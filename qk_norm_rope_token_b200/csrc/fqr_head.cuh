@@ -73,13 +73,18 @@ __device__ __forceinline__ int weight_slot(int e) {
 }
 
 // Stage both weight vectors (fp32, permuted) in s_w[0, 256); NULL -> ones.
-__device__ __forceinline__ void stage_weights(float* s_w, const uint16_t* qw, const uint16_t* kw) {
-  for (int i = threadIdx.x; i < 2 * kHeadDim; i += blockDim.x) {
-    const int e = i & (kHeadDim - 1);
-    const uint16_t* w = i < kHeadDim ? qw : kw;
-    const float v = w != nullptr ? __uint_as_float(static_cast<uint32_t>(w[e]) << 16) : 1.0f;
-    s_w[(i & kHeadDim) + weight_slot(e)] = v;
-  }
+// For blocks of at least 256 threads: weight_prefetch loads one value per
+// thread at kernel entry, weight_store writes it after the first round trip.
+__device__ __forceinline__ float weight_prefetch(const uint16_t* qw, const uint16_t* kw) {
+  const int i = threadIdx.x;
+  if (i >= 2 * kHeadDim) return 0.0f;
+  const uint16_t* w = i < kHeadDim ? qw : kw;
+  return w != nullptr ? __uint_as_float(static_cast<uint32_t>(__ldg(w + (i & (kHeadDim - 1)))) << 16)
+                      : 1.0f;
+}
+__device__ __forceinline__ void weight_store(float* s_w, float v) {
+  const int i = threadIdx.x;
+  if (i < 2 * kHeadDim) s_w[(i & kHeadDim) + weight_slot(i & (kHeadDim - 1))] = v;
 }
 
 __device__ __forceinline__ void unpack_pairs(uint4 xa, uint4 xb, float2* y) {
@@ -102,6 +107,27 @@ __device__ __forceinline__ uint2 pack_e4m3_pairs(const float2* y) {
                     pack_e4m3x2(y[2].x, y[2].y) | (pack_e4m3x2(y[3].x, y[3].y) << 16));
 }
 
+__device__ __forceinline__ float2 neg2(float2 v) { return make_float2(-v.x, -v.y); }
+
+// a / b for the dynamic Q payload, where the divisor b = q_scale is used for a
+// whole head and |a / b| <= upper_max <= 448 by construction.  Given
+// r = __frcp_rn(b): one correction step of Markstein's method (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): q0 = a r, e = a - b q0 (exact
+// with an FMA), q = q0 + e r -- written as -(-e r - q0) so that a zero
+// dividend keeps its sign.  Two lanes at once (f32x2).  Within that bounded
+// domain the E4M3 code of the result equals the code of IEEE a / b for every
+// a, and the quotient itself is bit-equal when |a| >= 2^-100 or a = +-0
+// (tests/test_gpu_division.py checks both over every binary32 dividend for a
+// set of q_scale values and over 2^33 random pairs).  Outside it -- |a / b|
+// beyond the float range -- the correction is not used.
+__device__ __forceinline__ float2 div2_bounded(float2 a, float2 b, float2 r) {
+  const float2 q0 = mul2(a, r);
+  const float2 e = fma2(neg2(q0), b, a);
+  return neg2(fma2(neg2(e), r, neg2(q0)));
+}
+
+// IEEE division of every value by d (K / V payloads: arbitrary scales).
 __device__ __forceinline__ void divide_pairs(float2* y, float d) {
 #pragma unroll
   for (int j = 0; j < 8; ++j) y[j] = make_float2(__fdiv_rn(y[j].x, d), __fdiv_rn(y[j].y, d));
@@ -134,13 +160,42 @@ __device__ __forceinline__ void zero_tail_column(char* page_base, int row0, int 
   }
 }
 
+// The cos/sin values lane l8 needs for its 8 pairs: NeoX (rot 128) pairs
+// (8l+k, 64+8l+k); GPT-J pairs 4l+j (chunk A) and 32+4l+j (chunk B), with
+// c = s = 0 outside the rotated dims (those pairs are not rotated).
+template <int STYLE, bool CS_SMEM>
+__device__ __forceinline__ void load_cs(const float* cs_row, int rot, int l8, float2* c,
+                                        float2* s) {
+  if (STYLE == 0) {
+    const float4 c0 = ld_cs4<CS_SMEM>(cs_row + 8 * l8);
+    const float4 c1 = ld_cs4<CS_SMEM>(cs_row + 8 * l8 + 4);
+    const float4 s0 = ld_cs4<CS_SMEM>(cs_row + 64 + 8 * l8);
+    const float4 s1 = ld_cs4<CS_SMEM>(cs_row + 68 + 8 * l8);
+    c[0] = make_float2(c0.x, c0.y); c[1] = make_float2(c0.z, c0.w);
+    c[2] = make_float2(c1.x, c1.y); c[3] = make_float2(c1.z, c1.w);
+    s[0] = make_float2(s0.x, s0.y); s[1] = make_float2(s0.z, s0.w);
+    s[2] = make_float2(s1.x, s1.y); s[3] = make_float2(s1.z, s1.w);
+  } else {
+    const int half = rot >> 1;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int ia = 4 * l8 + j, ib = 32 + 4 * l8 + j;
+      c[j].x = ia < half ? ld_cs1<CS_SMEM>(cs_row + ia) : 0.0f;
+      s[j].x = ia < half ? ld_cs1<CS_SMEM>(cs_row + half + ia) : 0.0f;
+      c[j].y = ib < half ? ld_cs1<CS_SMEM>(cs_row + ib) : 0.0f;
+      s[j].y = ib < half ? ld_cs1<CS_SMEM>(cs_row + half + ib) : 0.0f;
+    }
+  }
+}
+
 // Norm + RoPE + quantisation + store of head h of row r.  xa/xb: the lane's two
 // 16-byte slices of the packed head; cs_row: the row's fp32 [cos | sin]
 // (shared or global memory); s_w: staged weights.  gmask: the 8-lane group.
-template <int POLICY, int STYLE, bool CS_SMEM>
-__device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& r, int h,
-                                             uint4 xa, uint4 xb, const float* cs_row,
-                                             const float* s_w, int l8, unsigned gmask) {
+template <int POLICY, int STYLE>
+__device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCtx& r, int h,
+                                                uint4 xa, uint4 xb, const float2* c,
+                                                const float2* s, const float* s_w, int l8,
+                                                unsigned gmask) {
   constexpr int ES = POLICY == 0 ? 2 : 1;
   const int P = a.page_size;
   float2 y[8];
@@ -162,29 +217,6 @@ __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& 
   }
 
   const bool is_q = h < a.Hq;
-  // ------------------------------------------------------------ cos / sin
-  float2 c[4], s[4];
-  if (STYLE == 0) {  // NeoX, rot == 128: pair k of chunk A is (8l+k, 64+8l+k)
-    const float4 c0 = ld_cs4<CS_SMEM>(cs_row + 8 * l8);
-    const float4 c1 = ld_cs4<CS_SMEM>(cs_row + 8 * l8 + 4);
-    const float4 s0 = ld_cs4<CS_SMEM>(cs_row + 64 + 8 * l8);
-    const float4 s1 = ld_cs4<CS_SMEM>(cs_row + 68 + 8 * l8);
-    c[0] = make_float2(c0.x, c0.y); c[1] = make_float2(c0.z, c0.w);
-    c[2] = make_float2(c1.x, c1.y); c[3] = make_float2(c1.z, c1.w);
-    s[0] = make_float2(s0.x, s0.y); s[1] = make_float2(s0.z, s0.w);
-    s[2] = make_float2(s1.x, s1.y); s[3] = make_float2(s1.z, s1.w);
-  } else {  // GPT-J: y[j] is pair i = 4l + j (chunk A), y[4+j] pair 32 + 4l + j
-    const int half = a.rot >> 1;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int ia = 4 * l8 + j, ib = 32 + 4 * l8 + j;
-      c[j].x = ia < half ? ld_cs1<CS_SMEM>(cs_row + ia) : 0.0f;
-      s[j].x = ia < half ? ld_cs1<CS_SMEM>(cs_row + half + ia) : 0.0f;
-      c[j].y = ib < half ? ld_cs1<CS_SMEM>(cs_row + ib) : 0.0f;
-      s[j].y = ib < half ? ld_cs1<CS_SMEM>(cs_row + half + ib) : 0.0f;
-    }
-  }
-
   // -------------------------------------------------------------- RMSNorm
   if (is_q ? a.has_qw : a.has_kw) {
     float2 acc = make_float2(0.0f, 0.0f);
@@ -240,7 +272,10 @@ __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& 
       amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 1));
       const float qs = __fdiv_rn(fmaxf(amax, 1e-6f), a.upper_max);
       if (l8 == 0) a.q_scale[static_cast<int64_t>(r.t) * a.Hq + h] = qs;
-      divide_pairs(y, qs);
+      const float rq = __frcp_rn(qs);
+      const float2 b2 = make_float2(qs, qs), r2 = make_float2(rq, rq);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[j] = div2_bounded(y[j], b2, r2);
     } else if (POLICY == 2) {
       const float qsi = __ldg(a.q_scale_inv);
       const float2 qv = make_float2(qsi, qsi);
@@ -256,6 +291,17 @@ __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& 
     store_head<POLICY>(dst, y, l8);
     if (r.is_last) zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
   }
+}
+
+// As process_head_cs, loading the cos/sin values from cs_row first (V heads
+// need none).
+template <int POLICY, int STYLE, bool CS_SMEM>
+__device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& r, int h,
+                                             uint4 xa, uint4 xb, const float* cs_row,
+                                             const float* s_w, int l8, unsigned gmask) {
+  float2 c[4], s[4];
+  if (h < a.Hq + a.Hkv) load_cs<STYLE, CS_SMEM>(cs_row, a.rot, l8, c, s);
+  process_head_cs<POLICY, STYLE>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
 }
 
 // Zero the whole tail (rows [last+1, P), all heads) of request b's last page in
