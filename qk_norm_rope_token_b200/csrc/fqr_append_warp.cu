@@ -14,9 +14,10 @@
 //     the second dependent round trip overlaps the batch validation.
 //   * every block stages q_indptr / seq_lens in shared memory and validates the
 //     whole batch (stage_and_validate); a malformed batch writes only flags.
-//   * the K/V heads of a request's last new row also zero their column of the
-//     tail rows of that page; one "request task" per request zeroes the tail of
-//     requests that append nothing in this call.
+//   * the warps of a request's last new row split that request's last-page
+//     tail (both caches) evenly between them and store their share of zeros
+//     after their heads; one "request task" per request zeroes the tail of
+//     requests that append nothing.
 #include "fqr_head.cuh"
 #include "fqr_launch.h"
 
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
       r0.slot_row = p - pidx * a.hp.page_size;
       r0.pos = static_cast<int>(pos);
       r0.is_last = t0 == e_hi - 1;
-      if (h0 >= a.hp.Hq)
+      if (h0 >= a.hp.Hq || r0.is_last)  // K/V slot, or the tail share of the last row
         r0.page = __ldg(a.page_table + static_cast<int64_t>(gb) * a.max_pages + pidx);
       if (h0 < a.hp.Hq + a.hp.Hkv)
         load_cs<STYLE, false>(a.cs + pos * a.hp.rot, a.hp.rot, l8, c0, s0);
@@ -120,13 +121,14 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
     if (w < a.n_head) {
       const uint4 xa = pa, xb = pb;
       if (w + nwarps < a.n_head) warp_load_head(a, w + nwarps, g, l8, pa, pb);
+      const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
+      const int quad = w - t * a.quads;
       if (w == gwarp && early) {  // the batch is valid: the early lookups stand
-        process_head_cs<POLICY, STYLE>(a.hp, r0, h0, xa, xb, c0, s0, s_w, l8, gmask);
+        process_head_cs<POLICY, STYLE, false>(a.hp, r0, h0, xa, xb, c0, s0, s_w, l8, gmask);
+        if (r0.is_last) zero_tail_share(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane);
         continue;
       }
-      const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
-      const int h = (w - t * a.quads) * 4 + g;
-      if (h >= a.H) continue;  // the whole 8-lane group skips together
+      const int h = quad * 4 + g;
       const int b = request_of_row(s_indptr, a.B, t);
       const int end = s_indptr[b + 1];
       const int p_slot = t + s_seq[b] - end;
@@ -136,9 +138,14 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
       r.slot_row = p_slot - pidx * a.hp.page_size;
       r.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : p_slot;
       r.is_last = t == end - 1;
-      r.page = h >= a.hp.Hq ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx) : 0;
-      const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
-      process_head<POLICY, STYLE, false>(a.hp, r, h, xa, xb, cs_row, s_w, l8, gmask);
+      r.page = (h >= a.hp.Hq || r.is_last)
+                   ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx)
+                   : 0;
+      if (h < a.H) {  // (a group past the last head only helps with the tail)
+        const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
+        process_head<POLICY, STYLE, false, false>(a.hp, r, h, xa, xb, cs_row, s_w, l8, gmask);
+      }
+      if (r.is_last) zero_tail_share(a.hp, r.page, r.slot_row, quad, a.qdiv, lane);
     } else {
       const int b = w - a.n_head;  // request task: tail of a request without new rows
       const int L = s_seq[b];

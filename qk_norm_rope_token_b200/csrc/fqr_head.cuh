@@ -188,10 +188,30 @@ __device__ __forceinline__ void load_cs(const float* cs_row, int rot, int l8, fl
   }
 }
 
+// Zero share `part` of `parts` (pdiv divides by parts) of a request's tail
+// rows [last+1, P) in both caches -- the K span, then the V span, in 16-byte
+// units -- so that all the warps of the request's last row split it evenly.
+__device__ __forceinline__ void zero_tail_share(const HeadParams& a, int page, int last,
+                                                uint32_t part, const FastDiv& pdiv, int lane) {
+  const uint32_t span = static_cast<uint32_t>(a.page_size - 1 - last) * a.row_bytes;  // per cache
+  const uint32_t units = span / 8;                                                  // 2 * span / 16
+  const uint32_t u0 = pdiv.div(units * part), u1 = pdiv.div(units * (part + 1));
+  const int64_t beg = static_cast<int64_t>(last + 1) * a.row_bytes;
+  char* kb = a.k_cache + static_cast<int64_t>(page) * a.k_page_bytes + beg;
+  char* vb = a.v_cache + static_cast<int64_t>(page) * a.v_page_bytes + beg;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (uint32_t u = u0 + lane; u < u1; u += 32) {
+    const uint32_t o = u * 16;
+    st_v4(o < span ? kb + o : vb + (o - span), z);
+  }
+}
+
 // Norm + RoPE + quantisation + store of head h of row r.  xa/xb: the lane's two
 // 16-byte slices of the packed head; cs_row: the row's fp32 [cos | sin]
 // (shared or global memory); s_w: staged weights.  gmask: the 8-lane group.
-template <int POLICY, int STYLE>
+// TAILS: the K/V heads of a request's last row also zero their column of the
+// tail rows (when the caller does not split the tail over warps itself).
+template <int POLICY, int STYLE, bool TAILS = true>
 __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCtx& r, int h,
                                                 uint4 xa, uint4 xb, const float2* c,
                                                 const float2* s, const float* s_w, int l8,
@@ -212,7 +232,7 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
       divide_pairs(y, __ldg(a.v_scale));
       store_head<POLICY>(dst, y, l8);
     }
-    if (r.is_last) zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
+    if (TAILS && r.is_last) zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
     return;
   }
 
@@ -289,19 +309,19 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
     char* dst = page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
     if (POLICY != 0) divide_pairs(y, __ldg(a.k_scale));
     store_head<POLICY>(dst, y, l8);
-    if (r.is_last) zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
+    if (TAILS && r.is_last) zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
   }
 }
 
 // As process_head_cs, loading the cos/sin values from cs_row first (V heads
 // need none).
-template <int POLICY, int STYLE, bool CS_SMEM>
+template <int POLICY, int STYLE, bool CS_SMEM, bool TAILS = true>
 __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& r, int h,
                                              uint4 xa, uint4 xb, const float* cs_row,
                                              const float* s_w, int l8, unsigned gmask) {
   float2 c[4], s[4];
   if (h < a.Hq + a.Hkv) load_cs<STYLE, CS_SMEM>(cs_row, a.rot, l8, c, s);
-  process_head_cs<POLICY, STYLE>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+  process_head_cs<POLICY, STYLE, TAILS>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
 }
 
 // Zero the whole tail (rows [last+1, P), all heads) of request b's last page in
