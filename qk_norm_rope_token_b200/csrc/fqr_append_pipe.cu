@@ -173,7 +173,10 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
 template <int POLICY, int STYLE, bool CSB>
 __device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t* full,
                         uint64_t* empty, const float* s_w, int64_t u0, int nunits) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // (a shuffled warp index is known to the compiler to be warp-uniform, so the
+  // quad loop below and the kind dispatch inside it branch uniformly)
+  const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
+  const int lane = threadIdx.x & 31;
   const int g = lane >> 3, l8 = lane & 7;
   const unsigned gmask = 0xFFu << (8 * g);
   const int S = a.stages;
@@ -199,15 +202,14 @@ __device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t
     if (q < 0) q += kConsumers;
     for (; q < nq; q += kConsumers) {
       const int hl = 4 * q + g;
+      uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = xa;
       if (hl < nh) {
         const unsigned char* src = st + 16 + a.cs_bytes + hl * (kHeadDim * 2) + 16 * l8;
-        if (CSB)
-          process_head<POLICY, STYLE, true>(a.hp, r, h0 + hl, ld_smem_v4(src),
-                                            ld_smem_v4(src + 128), cs_row, s_w, l8, gmask);
-        else
-          process_head<POLICY, STYLE, false>(a.hp, r, h0 + hl, ld_smem_v4(src),
-                                             ld_smem_v4(src + 128), cs_row, s_w, l8, gmask);
+        xa = ld_smem_v4(src);
+        xb = ld_smem_v4(src + 128);
       }
+      process_quad<POLICY, STYLE, CSB>(a.hp, r, h0 + 4 * q, h0 + nh, g, xa, xb, cs_row, s_w, l8,
+                                       gmask);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -236,6 +238,8 @@ __device__ void zero_empty_request_tails(const PipeArgs& a, const int* s_indptr,
   }
 }
 
+// Two resident blocks per SM: 18 warps, at most 5 on each of the 4 sub-partition
+// register files (16K registers each), so at most 96 registers a thread.
 template <int POLICY, int STYLE>
 __global__ void __launch_bounds__(kPipeThreads, 2) pipe_append_kernel(const PipeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];

@@ -59,7 +59,10 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   int* s_indptr = smem + 2 * kHeadDim;          // B + 1
   int* s_seq = s_indptr + a.B + 1;              // B
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // (a shuffled warp index is known to the compiler to be warp-uniform, so
+  // the task loop and the head-kind dispatch branch uniformly)
+  const int lane = threadIdx.x & 31;
+  const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
   const int g = lane >> 3, l8 = lane & 7;
   const unsigned gmask = 0xFFu << (8 * g);
   const int gwarp = blockIdx.x * kWarps + warp;
@@ -124,7 +127,8 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
       const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
       const int quad = w - t * a.quads;
       if (w == gwarp && early) {  // the batch is valid: the early lookups stand
-        process_head_cs<POLICY, STYLE, false>(a.hp, r0, h0, xa, xb, c0, s0, s_w, l8, gmask);
+        process_quad_cs<POLICY, STYLE, false>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, s_w, l8,
+                                              gmask);
         if (r0.is_last) zero_tail_share(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane);
         continue;
       }
@@ -141,10 +145,10 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
       r.page = (h >= a.hp.Hq || r.is_last)
                    ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx)
                    : 0;
-      if (h < a.H) {  // (a group past the last head only helps with the tail)
-        const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
-        process_head<POLICY, STYLE, false, false>(a.hp, r, h, xa, xb, cs_row, s_w, l8, gmask);
-      }
+      // (a group past the last head only helps with the tail)
+      const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
+      process_quad<POLICY, STYLE, false, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, s_w, l8,
+                                                gmask);
       if (r.is_last) zero_tail_share(a.hp, r.page, r.slot_row, quad, a.qdiv, lane);
     } else {
       const int b = w - a.n_head;  // request task: tail of a request without new rows

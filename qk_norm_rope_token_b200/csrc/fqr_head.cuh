@@ -117,20 +117,39 @@ __device__ __forceinline__ float2 neg2(float2 v) { return make_float2(-v.x, -v.y
 // with an FMA), q = q0 + e r -- written as -(-e r - q0) so that a zero
 // dividend keeps its sign.  Two lanes at once (f32x2).  Within that bounded
 // domain the E4M3 code of the result equals the code of IEEE a / b for every
-// a, and the quotient itself is bit-equal when |a| >= 2^-100 or a = +-0
-// (tests/test_gpu_division.py checks both over every binary32 dividend for a
-// set of q_scale values and over 2^33 random pairs).  Outside it -- |a / b|
-// beyond the float range -- the correction is not used.
+// a, and the quotient itself is bit-equal when a = +-0, or |a| >= 2^-100 and
+// the quotient is not subnormal (the theorem assumes no underflow; a
+// subnormal quotient encodes to a zero code either way).
+// tests/test_gpu_division.py checks both over every binary32 dividend for a
+// set of q_scale values and over 2^33 random pairs.  Outside the domain --
+// |a / b| beyond the float range -- the correction is not used.
 __device__ __forceinline__ float2 div2_bounded(float2 a, float2 b, float2 r) {
   const float2 q0 = mul2(a, r);
   const float2 e = fma2(neg2(q0), b, a);
   return neg2(fma2(neg2(e), r, neg2(q0)));
 }
 
-// IEEE division of every value by d (K / V payloads: arbitrary scales).
+// K / V payloads: every value divided by d (k_scale or v_scale, one value for
+// the whole call), then encoded to E4M3.  The lane's 16 quotients come from
+// div2_bounded when the division cannot overflow or lose the exactness of the
+// residual anywhere it matters -- 2^-80 <= d <= 2^80 and max|x| / d < 2^100
+// -- which makes every E4M3 code equal to the code of the IEEE quotient
+// (tests/test_gpu_division.py checks it over every binary32 dividend for a set
+// of scales).  A negative scale would give a zero quotient the wrong sign in
+// the correction; it, like any lane outside the guard, divides with __fdiv_rn.
 __device__ __forceinline__ void divide_pairs(float2* y, float d) {
+  const float r = __frcp_rn(d);
+  float m = 0.0f;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) y[j] = make_float2(__fdiv_rn(y[j].x, d), __fdiv_rn(y[j].y, d));
+  for (int j = 0; j < 8; ++j) m = fmaxf(m, fmaxf(fabsf(y[j].x), fabsf(y[j].y)));
+  if (d >= 0x1p-80f && d <= 0x1p80f && m * r < 0x1p100f) {
+    const float2 b2 = make_float2(d, d), r2 = make_float2(r, r);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = div2_bounded(y[j], b2, r2);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = make_float2(__fdiv_rn(y[j].x, d), __fdiv_rn(y[j].y, d));
+  }
 }
 
 // Store a head (16 values per lane) into a KV slot / out_q row at `dst`
@@ -206,12 +225,27 @@ __device__ __forceinline__ void zero_tail_share(const HeadParams& a, int page, i
   }
 }
 
+// What the 4 heads of a quad are, when the whole quad is known to be of one
+// kind (a warp-uniform value, so the per-head code has no divergent branch
+// on the head type); kAnyHead decides per head.
+enum HeadKind { kAnyHead = 0, kQHead = 1, kKHead = 2, kVHead = 3 };
+
+// Kind of heads [h0, h0 + 4) (all of them exist).
+__device__ __forceinline__ int quad_kind(const HeadParams& a, int h0) {
+  const int qk = a.Hq + a.Hkv;
+  if (h0 + 4 <= a.Hq) return kQHead;
+  if (h0 >= a.Hq && h0 + 4 <= qk) return kKHead;
+  if (h0 >= qk) return kVHead;
+  return kAnyHead;
+}
+
 // Norm + RoPE + quantisation + store of head h of row r.  xa/xb: the lane's two
 // 16-byte slices of the packed head; cs_row: the row's fp32 [cos | sin]
 // (shared or global memory); s_w: staged weights.  gmask: the 8-lane group.
 // TAILS: the K/V heads of a request's last row also zero their column of the
 // tail rows (when the caller does not split the tail over warps itself).
-template <int POLICY, int STYLE, bool TAILS = true>
+// KIND: the head's kind when the caller knows it (HeadKind).
+template <int POLICY, int STYLE, bool TAILS = true, int KIND = kAnyHead>
 __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCtx& r, int h,
                                                 uint4 xa, uint4 xb, const float2* c,
                                                 const float2* s, const float* s_w, int l8,
@@ -221,7 +255,8 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
   float2 y[8];
   unpack_pairs(xa, xb, y);
 
-  if (h >= a.Hq + a.Hkv) {  // ------------------------------------------ V
+  const bool is_v = KIND == kVHead || (KIND == kAnyHead && h >= a.Hq + a.Hkv);
+  if (is_v) {  // -------------------------------------------------------- V
     const int kh = h - a.Hq - a.Hkv;
     char* page_base = a.v_cache + static_cast<int64_t>(r.page) * a.v_page_bytes;
     char* dst = page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
@@ -236,7 +271,7 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
     return;
   }
 
-  const bool is_q = h < a.Hq;
+  const bool is_q = KIND == kQHead || (KIND == kAnyHead && h < a.Hq);
   // -------------------------------------------------------------- RMSNorm
   if (is_q ? a.has_qw : a.has_kw) {
     float2 acc = make_float2(0.0f, 0.0f);
@@ -246,7 +281,10 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
     ss += __shfl_xor_sync(gmask, ss, 4);
     ss += __shfl_xor_sync(gmask, ss, 2);
     ss += __shfl_xor_sync(gmask, ss, 1);
-    const float inv = __frcp_rn(__fsqrt_rn(__fadd_rn(ss * (1.0f / kHeadDim), a.eps)));
+    // rsqrtf: at most 2 ulp from 1/sqrt (CUDA's documented bound), against
+    // the correctly rounded sqrt then reciprocal of the step-wise definition;
+    // the parity bar propagates the difference with that of the summation order
+    const float inv = rsqrtf(__fadd_rn(ss * (1.0f / kHeadDim), a.eps));
     const float2 iv = make_float2(inv, inv);
     const float* wv = s_w + (is_q ? 0 : kHeadDim) + 4 * l8;
     const float4 w0 = lds_f4(wv);
@@ -315,13 +353,53 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
 
 // As process_head_cs, loading the cos/sin values from cs_row first (V heads
 // need none).
-template <int POLICY, int STYLE, bool CS_SMEM, bool TAILS = true>
+template <int POLICY, int STYLE, bool CS_SMEM, bool TAILS = true, int KIND = kAnyHead>
 __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& r, int h,
                                              uint4 xa, uint4 xb, const float* cs_row,
                                              const float* s_w, int l8, unsigned gmask) {
   float2 c[4], s[4];
-  if (h < a.Hq + a.Hkv) load_cs<STYLE, CS_SMEM>(cs_row, a.rot, l8, c, s);
-  process_head_cs<POLICY, STYLE, TAILS>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+  if (KIND == kQHead || KIND == kKHead || (KIND == kAnyHead && h < a.Hq + a.Hkv))
+    load_cs<STYLE, CS_SMEM>(cs_row, a.rot, l8, c, s);
+  process_head_cs<POLICY, STYLE, TAILS, KIND>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+}
+
+// process_head_cs for one quad whose first head is h0 (warp-uniform), with
+// the cos/sin values already loaded; see process_quad.
+template <int POLICY, int STYLE, bool TAILS = true>
+__device__ __forceinline__ void process_quad_cs(const HeadParams& a, const RowCtx& r, int h0,
+                                                int nheads, int g, uint4 xa, uint4 xb,
+                                                const float2* c, const float2* s,
+                                                const float* s_w, int l8, unsigned gmask) {
+  const int h = h0 + g;
+  const int kind = h0 + 4 <= nheads ? quad_kind(a, h0) : kAnyHead;
+  if (kind == kQHead)
+    process_head_cs<POLICY, STYLE, TAILS, kQHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+  else if (kind == kKHead)
+    process_head_cs<POLICY, STYLE, TAILS, kKHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+  else if (kind == kVHead)
+    process_head_cs<POLICY, STYLE, TAILS, kVHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+  else if (h < nheads)
+    process_head_cs<POLICY, STYLE, TAILS, kAnyHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+}
+
+// process_head for one quad whose first head is h0 (warp-uniform): the kind
+// is decided once for the warp when all four heads exist; otherwise each
+// group decides for its own head (h0 + g < nheads).
+template <int POLICY, int STYLE, bool CS_SMEM, bool TAILS = true>
+__device__ __forceinline__ void process_quad(const HeadParams& a, const RowCtx& r, int h0,
+                                             int nheads, int g, uint4 xa, uint4 xb,
+                                             const float* cs_row, const float* s_w, int l8,
+                                             unsigned gmask) {
+  const int h = h0 + g;
+  const int kind = h0 + 4 <= nheads ? quad_kind(a, h0) : kAnyHead;
+  if (kind == kQHead)
+    process_head<POLICY, STYLE, CS_SMEM, TAILS, kQHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+  else if (kind == kKHead)
+    process_head<POLICY, STYLE, CS_SMEM, TAILS, kKHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+  else if (kind == kVHead)
+    process_head<POLICY, STYLE, CS_SMEM, TAILS, kVHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+  else if (h < nheads)
+    process_head<POLICY, STYLE, CS_SMEM, TAILS, kAnyHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
 }
 
 // Zero the whole tail (rows [last+1, P), all heads) of request b's last page in

@@ -78,10 +78,12 @@ def changed_pages(after: torch.Tensor, before: torch.Tensor, chunk=2048) -> set:
 U32 = 2.0 ** -24
 # Relative bound on the difference of the RMSNorm output y between two fp32
 # evaluations that sum the 128 squares in different orders (sequential: gamma_127,
-# 16-term lanes + 3-level tree: gamma_18; halved by the square root; plus the
-# roundings of +eps, sqrt, 1/x and the two products): see the parity section of
-# the design notes.  The rotation then adds at most 2 u of each product term.
-K_COND = 85.0
+# 16-term lanes + 3-level tree: gamma_18; halved by the square root), plus the
+# roundings of +eps and the two products on each side, the correctly rounded
+# sqrt and 1/x of the definition (u each) and the kernel's rsqrtf (at most 2
+# ulp, 4 u): see the parity section of the design notes.  The rotation then
+# adds at most 2 u of each product term.
+K_COND = 87.0
 
 
 def _spacing_bf16(v):

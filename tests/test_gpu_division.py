@@ -1,8 +1,11 @@
-"""GPU check of the dynamic-Q payload division (one Markstein correction on a
-correctly rounded reciprocal) against IEEE division: bit-equal quotients for
-|a| >= 2^-100 or a = +-0, and equal E4M3 codes wherever |a / b| <= 448, over
+"""GPU checks of the payload divisions (one Markstein correction on a correctly
+rounded reciprocal) against IEEE division.  Dynamic Q: bit-equal quotients for
+a = +-0 or |a| >= 2^-100 with a normal quotient, and equal E4M3 codes
+wherever |a / b| <= 448, over
 every binary32 dividend for divisors across the q_scale range and over 2^33
-random pairs."""
+random pairs.  K / V (guarded, any value and scale): equal E4M3 codes over
+every binary32 dividend for a set of scales, inside and outside the guard, and
+over 2^32 random lanes of 16 mixed values."""
 import os
 import subprocess
 
@@ -37,4 +40,22 @@ def test_every_dividend(checker, bits):
 @pytest.mark.parametrize("seed", [1, 2])
 def test_random_pairs(checker, seed):
     r = subprocess.run([checker, "rand", str(seed), str(1 << 32)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
+# K / V scales: 0.05 and 0.02 (the workloads' scales), 1, a significand of all
+# ones, the guard's ends 2^-80 and 2^80, and 1e-30, 1e30 and -0.05 (outside
+# it: IEEE division)
+KV_SCALES = ["3d4ccccd", "3ca3d70a", "3f800000", "3f7fffff", "17800000", "67800000",
+             "0da24260", "7149f2ca", "bd4ccccd"]
+
+
+@pytest.mark.parametrize("bits", KV_SCALES)
+def test_kv_every_dividend(checker, bits):
+    r = subprocess.run([checker, "kvall", bits], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
+def test_kv_random_lanes(checker):
+    r = subprocess.run([checker, "kvrand", "3", str(1 << 32)], capture_output=True, text=True)
     assert r.returncode == 0, r.stdout + r.stderr
