@@ -42,8 +42,10 @@ extern "C" {
 #define FQR_HEAD_DIM 128
 
 /* fqr_append_params.schedule: how rows are spread over the GPU (the results
- * are identical).  AUTO picks LATENCY for small batches (decode) and
- * STREAMING for large ones (prefill). */
+ * are identical).  AUTO picks LATENCY while every warp task of it (one per
+ * 4 heads of a row, plus one per request) has a resident warp of its own --
+ * small batches such as decode -- and STREAMING beyond that (large decode
+ * batches, prefill). */
 #define FQR_SCHEDULE_AUTO 0
 #define FQR_SCHEDULE_LATENCY 1
 #define FQR_SCHEDULE_STREAMING 2

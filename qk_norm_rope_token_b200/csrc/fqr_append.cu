@@ -13,9 +13,6 @@
 
 namespace fqr {
 
-// Rows per SM from which the streaming schedule takes over in auto mode.
-constexpr int kStreamRowsPerSm = 4;
-
 int launch_append(const fqr_append_params& p, cudaStream_t stream) {
   HeadParams hp;
   const int es = p.quant_policy == 0 ? 2 : 1;
@@ -41,13 +38,12 @@ int launch_append(const fqr_append_params& p, cudaStream_t stream) {
 
   int schedule = p.schedule;
   if (schedule == FQR_SCHEDULE_AUTO) {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return FQR_ECUDA;
-    schedule = static_cast<int64_t>(p.T) >= static_cast<int64_t>(kStreamRowsPerSm) * sms
-                   ? FQR_SCHEDULE_STREAMING
-                   : FQR_SCHEDULE_LATENCY;
+    // latency while every warp task has a resident warp of its own (one
+    // pass, no task waits for another); streaming once the tasks outnumber
+    // the resident warps and a pipeline hides the rest
+    const int64_t cap = latency_capacity(p);
+    if (cap < 0) return FQR_ECUDA;
+    schedule = latency_tasks(p) <= cap ? FQR_SCHEDULE_LATENCY : FQR_SCHEDULE_STREAMING;
   }
   return schedule == FQR_SCHEDULE_STREAMING ? launch_append_pipe(p, hp, stream)
                                             : launch_append_warp(p, hp, stream);

@@ -172,6 +172,30 @@ static WarpKernel select_warp(int policy, int style) {
   return warp_append_kernel<2, 1>;
 }
 
+static size_t warp_smem(const fqr_append_params& p) {
+  return static_cast<size_t>(2 * kHeadDim + 2 * p.B + 1) * sizeof(int);
+}
+
+int64_t latency_tasks(const fqr_append_params& p) {
+  return static_cast<int64_t>(p.T) * ((p.Hq + 2 * p.Hkv + 3) / 4) + p.B;
+}
+
+int64_t latency_capacity(const fqr_append_params& p) {
+  int dev = 0, sms = 0, per_sm = 0;
+  const void* fn = reinterpret_cast<const void*>(select_warp(p.quant_policy, p.rope_style));
+  const size_t smem = warp_smem(p);
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return -1;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return -1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem) != cudaSuccess)
+    return -1;
+  return static_cast<int64_t>(per_sm) * sms * kWarps;
+}
+
 int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream) {
   WarpArgs a;
   a.hp = hp;
@@ -195,7 +219,7 @@ int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStr
   a.page_table = p.page_table;
   a.max_pages = p.max_pages;
   a.flags = p.flags;
-  const size_t smem = static_cast<size_t>(2 * kHeadDim + 2 * p.B + 1) * sizeof(int);
+  const size_t smem = warp_smem(p);
   WarpKernel k = select_warp(p.quant_policy, p.rope_style);
   return launch_persistent(reinterpret_cast<const void*>(k), n_head + p.B, smem, stream,
                            [&](int grid) { return launch_pdl(k, grid, kThreads, smem, stream, a); });

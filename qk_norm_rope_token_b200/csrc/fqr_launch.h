@@ -13,6 +13,10 @@ namespace fqr {
 struct HeadParams;
 int launch_append(const fqr_append_params& p, cudaStream_t stream);
 int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream);
+// Warp tasks of the latency schedule for p, and how many warps of it the
+// device holds at once (-1 if the runtime cannot tell).
+int64_t latency_tasks(const fqr_append_params& p);
+int64_t latency_capacity(const fqr_append_params& p);
 int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream);
 int launch_mla(const fqr_mla_params& p, cudaStream_t stream);
 
