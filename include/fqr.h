@@ -53,6 +53,12 @@ extern "C" {
  * is staged in shared memory by every thread block. */
 #define FQR_MAX_BATCH 16384
 
+/* fqr_append_params.norm_style: how the bf16 norm weight w scales the
+ * normalised value.  RMS: y = x_hat * w.  GEMMA: y = x_hat * (1 + w), with
+ * 1 + w formed in fp32 (Gemma-style QK norm, TensorRT-LLM PR #16024). */
+#define FQR_NORM_RMS 0
+#define FQR_NORM_GEMMA 1
+
 /*
  * fqr_append_paged -- per-head Q/K RMSNorm, RoPE, optional FP8 E4M3
  * quantisation, and the paged K/V append with last-page tail zeroing.
@@ -69,29 +75,40 @@ extern "C" {
  * and goes to slot (page_table[b, p_r / P], p_r % P) of both caches.  RoPE
  * uses positions[r] when `positions` is given, else p_r.  In fp32:
  *     y = x * (1/sqrt(sum(x^2)/128 + eps)) * w         (Q heads with q_norm_w,
- *                                                       K heads with k_norm_w)
+ *                                                       K heads with k_norm_w;
+ *                                       w -> 1 + w for norm_style GEMMA)
  *     NeoX:  (y_i, y_{i+64})  -> (y_i c_i - y_{i+64} s_i, y_{i+64} c_i + y_i s_i)
  *     GPT-J: (y_2i, y_2i+1)   -> (y_2i c_i - y_2i+1 s_i, y_2i+1 c_i + y_2i s_i)
  *            with c_i = cos_sin[pos, i], s_i = cos_sin[pos, rot_dim/2 + i];
  *            dims >= rot_dim pass through.
  * Outputs by quant_policy:
  *     0: out_q = bf16(q); K = bf16(k); V = the input bits (BF16 caches)
- *     1: q_scale[r,h] = max(max_i |q_i|, 1e-6) / upper_max,
- *        out_q = e4m3(q / q_scale[r,h]); K = e4m3(k / *k_scale);
+ *     1: s = max(max_i |q_i|, 1e-6) / upper_max for each (row, Q head),
+ *        out_q = e4m3(q / s); K = e4m3(k / *k_scale);
  *        V = e4m3(v / *v_scale)                            (FP8 caches)
+ *        s is stored in q_scale, by layout:
+ *          max_seqlen == 0 (decode):  q_scale[r, h]         fp32 [T, Hq]
+ *          max_seqlen  > 0 (prefill): q_scale[b, h, r - q_indptr[b]]
+ *                              fp32 [B, Hq, round_up(max_seqlen, 128)];
+ *          entries past a request's rows are not written.
  *     2: out_q = e4m3(q * *q_scale_inv); K, V as in policy 1
  * (e4m3 = round to nearest even, saturating at +-448; bf16 = RNE).
  * Then, for every request with L_b > 0, rows [(L_b-1) % P + 1, P) of page
  * page_table[b, (L_b-1) / P] are zeroed in both caches.
+ * With out_k / out_v given, the K and V payloads go to row r of those
+ * caller-owned buffers instead: the paged caches and the page table are not
+ * used (they may be NULL), no slot is written and no tail is zeroed (the
+ * FlashInfer PR #5956 review: redirected K/V writes leave the caches alone).
  *
  * flags[b] = 0 after a valid call (requests without new tokens included).
  * flags[b] = -2 (all flags) only if the kernel gave up waiting for its own
  * shared-memory copies (a bounded wait that should never expire).
  * If the metadata is malformed -- q_indptr[0] != 0, q_indptr[B] != T, any
- * q_indptr decrease, L_b < n_b, L_b > max_pages * P, or (derived positions)
- * L_b > cos_sin_rows, or (explicit positions) any position outside
- * [0, cos_sin_rows) -- then EVERY flag is set to -1 and nothing else is
- * written: no out_q, q_scale or cache byte.  The check runs on the device
+ * q_indptr decrease, L_b < n_b, L_b > max_pages * P (paged caches only), or
+ * (derived positions) L_b > cos_sin_rows, or (explicit positions) any
+ * position outside [0, cos_sin_rows), or (policy 1 with max_seqlen > 0)
+ * n_b > max_seqlen -- then EVERY flag is set to -1 and nothing else is
+ * written: no out_q, q_scale, out_k, out_v or cache byte.  The check runs on the device
  * inside the same launch (no host sync), so the call can be captured in a
  * CUDA graph and replayed.  Read the flags after the stream completes.
  *
@@ -144,6 +161,16 @@ typedef struct fqr_append_params {
   float* q_scale;
   int32_t* flags;
   int32_t schedule;           /* FQR_SCHEDULE_*; 0 = automatic                */
+  /* policy 1: 0 = decode q_scale layout [T, Hq]; > 0 = prefill layout
+   * [B, Hq, round_up(max_seqlen, 128)] and the n_b <= max_seqlen check.
+   * Ignored by policies 0 and 2.  >= 0;
+   * B * Hq * round_up(max_seqlen, 128) < 2^31. */
+  int32_t max_seqlen;
+  int32_t norm_style;         /* FQR_NORM_RMS or FQR_NORM_GEMMA               */
+  /* optional caller-owned K / V outputs [T, Hkv, 128] (the cache element
+   * type), 16-byte aligned, both or neither; NULL = the paged caches */
+  void* out_k;
+  void* out_v;
 } fqr_append_params;
 
 int fqr_append_paged(const fqr_append_params* p, void* stream);

@@ -37,6 +37,7 @@ class _AppendArgs(ctypes.Structure):
         ("k_cache", c_vp), ("v_cache", c_vp),
         ("k_page_stride", c_i64), ("v_page_stride", c_i64),
         ("out_q", c_vp), ("q_scale", c_vp), ("flags", c_vp),
+        ("max_seqlen", c_i32), ("norm_style", c_i32), ("out_k", c_vp), ("out_v", c_vp),
     ]
 
 
@@ -69,7 +70,8 @@ def lib() -> ctypes.CDLL:
         L.fqro_rmsnorm.argtypes = [c_vp, c_vp, ctypes.c_int, c_f32, c_vp]
         L.fqro_rope_neox.argtypes = [c_vp, c_vp, ctypes.c_int]
         L.fqro_rope_gptj.argtypes = [c_vp, c_vp, ctypes.c_int]
-        L.fqro_validate.argtypes = [c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp]
+        L.fqro_validate.argtypes = [c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp,
+                                    c_i32, c_i32]
         L.fqro_validate.restype = ctypes.c_int
         L.fqro_append_paged.argtypes = [ctypes.POINTER(_AppendArgs)]
         L.fqro_append_paged.restype = ctypes.c_int
@@ -127,35 +129,48 @@ def rope(y, cs_row, style: int) -> np.ndarray:
 
 
 def validate(q_indptr, seq_lens, T, max_pages, page_size, cos_sin_rows,
-             positions=None) -> int:
+             positions=None, max_seqlen=0, paged=True) -> int:
     q_indptr = np.ascontiguousarray(q_indptr, dtype=np.int32)
     seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
     pos = None if positions is None else np.ascontiguousarray(positions, dtype=np.int64)
     return lib().fqro_validate(_ptr(q_indptr), _ptr(seq_lens), len(seq_lens), T,
-                               max_pages, page_size, cos_sin_rows, _ptr(pos))
+                               max_pages, page_size, cos_sin_rows, _ptr(pos),
+                               max_seqlen, 1 if paged else 0)
 
 
 # ---------------------------------------------------------------- methods --
 
 def new_outputs(w):
-    """Output buffers of the append, pre-filled with sentinels."""
+    """Output buffers of the append, pre-filled with sentinels (q_scale in the
+    workload's layout)."""
     qdt = np.uint16 if w.quant_policy == 0 else np.uint8
     out_q = np.full((w.T, w.Hq, 128), 0xFF, dtype=qdt)
-    q_scale = np.full((w.T, w.Hq), np.nan, dtype=np.float32)
+    q_scale = np.full(w.q_scale_shape, np.nan, dtype=np.float32)
     flags = np.full((w.B,), 0x5A5A5A5A, dtype=np.int32)
     return out_q, q_scale, flags
+
+
+def new_kv_outputs(w):
+    """Caller-owned K / V outputs [T, Hkv, 128] (cache element type),
+    pre-filled with sentinels."""
+    dt = np.uint16 if w.quant_policy == 0 else np.uint8
+    return (np.full((w.T, w.Hkv, 128), 0xEE, dtype=dt),
+            np.full((w.T, w.Hkv, 128), 0xDD, dtype=dt))
 
 
 def append_paged(w, k_cache: np.ndarray, v_cache: np.ndarray, out_q: np.ndarray,
                  q_scale: Optional[np.ndarray], flags: np.ndarray, *,
                  page_table: Optional[np.ndarray] = None,
                  q_indptr: Optional[np.ndarray] = None,
-                 seq_lens: Optional[np.ndarray] = None) -> int:
+                 seq_lens: Optional[np.ndarray] = None,
+                 out_k: Optional[np.ndarray] = None,
+                 out_v: Optional[np.ndarray] = None) -> int:
     """Run the oracle append on host caches [n_pages, page_size, Hkv, 128].
 
     `page_table`, `q_indptr` and `seq_lens` override the workload's arrays
     (used to remap pages into a compact host cache, or to plant malformed
-    metadata)."""
+    metadata).  With out_k / out_v ([T, Hkv, 128]) the K/V payloads go there
+    and the caches are left alone."""
     pt = np.ascontiguousarray(w.page_table if page_table is None else page_table,
                               dtype=np.int32)
     ind = np.ascontiguousarray(w.q_indptr if q_indptr is None else q_indptr, dtype=np.int32)
@@ -177,7 +192,9 @@ def append_paged(w, k_cache: np.ndarray, v_cache: np.ndarray, out_q: np.ndarray,
         k_cache=_ptr(k_cache), v_cache=_ptr(v_cache),
         k_page_stride=int(np.prod(k_cache.shape[1:])),
         v_page_stride=int(np.prod(v_cache.shape[1:])),
-        out_q=_ptr(out_q), q_scale=_ptr(q_scale), flags=_ptr(flags))
+        out_q=_ptr(out_q), q_scale=_ptr(q_scale), flags=_ptr(flags),
+        max_seqlen=w.max_seqlen, norm_style=w.norm_style,
+        out_k=_ptr(out_k), out_v=_ptr(out_v))
     return lib().fqro_append_paged(ctypes.byref(a))
 
 
@@ -211,4 +228,4 @@ def concat_mla_cache(w, q: np.ndarray, latent: np.ndarray, flags: np.ndarray, *,
 
 
 __all__ = ["lib", "e4m3", "bf16", "bf16_to_f32", "rmsnorm", "rope", "validate",
-           "new_outputs", "append_paged", "concat_mla_cache"]
+           "new_outputs", "new_kv_outputs", "append_paged", "concat_mla_cache"]

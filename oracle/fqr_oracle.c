@@ -160,15 +160,18 @@ static void rope(float* y, const float* cs_row, int rot, int style) {
 /* ------------------------------------------------------------------------ */
 int fqro_validate(const int32_t* q_indptr, const int32_t* seq_lens, int32_t B,
                   int32_t T, int32_t max_pages, int32_t page_size,
-                  int32_t cos_sin_rows, const int64_t* positions) {
+                  int32_t cos_sin_rows, const int64_t* positions,
+                  int32_t max_seqlen, int32_t paged) {
   if (q_indptr[0] != 0) return 1;
   if (q_indptr[B] != T) return 1;
   for (int32_t b = 0; b < B; ++b) {
     int64_t lo = q_indptr[b], hi = q_indptr[b + 1], L = seq_lens[b];
     if (hi < lo) return 1;
     if (L < hi - lo) return 1;  /* derived positions would go negative */
-    if (L > (int64_t)max_pages * page_size) return 1;
+    if (paged && L > (int64_t)max_pages * page_size) return 1;
     if (!positions && L > cos_sin_rows) return 1;
+    /* dynamic-Q prefill: a request may not outgrow its q_scale rows */
+    if (max_seqlen > 0 && hi - lo > max_seqlen) return 1;
   }
   if (positions) {
     for (int32_t t = 0; t < T; ++t)
@@ -185,17 +188,30 @@ static void widen_head(const uint16_t* src, float* x, int n) {
   for (int i = 0; i < n; ++i) x[i] = fqro_bf16_to_f32(src[i]);
 }
 
+/* Norm weights as fp32; the Gemma-style norm scales by 1 + w, formed in fp32
+ * ([TRT] "qk_norm_use_gemma"). */
+static void norm_weights(const uint16_t* w, int gemma, float* out) {
+  widen_head(w, out, D);
+  if (gemma)
+    for (int i = 0; i < D; ++i) out[i] = 1.0f + out[i];
+}
+
 int fqro_append_paged(const fqro_append_args* a) {
+  /* the dynamic-Q prefill layout and its max_seqlen check exist for policy 1
+   * only; with caller-owned K/V outputs no page is addressed */
+  const int32_t msl = a->quant_policy == 1 ? a->max_seqlen : 0;
+  const int paged = a->out_k == NULL;
   if (fqro_validate(a->q_indptr, a->seq_lens, a->B, a->T, a->max_pages,
-                    a->page_size, a->cos_sin_rows, a->positions)) {
+                    a->page_size, a->cos_sin_rows, a->positions, msl, paged)) {
     for (int32_t b = 0; b < a->B; ++b) a->flags[b] = -1;
     return 1;
   }
   const int P = a->page_size;
   const int fp8 = a->quant_policy != 0;
+  const int64_t ld = ((int64_t)msl + 127) / 128 * 128;  /* prefill q_scale row */
   float wq[D], wk[D], x[D], y[D];
-  if (a->q_norm_w) widen_head(a->q_norm_w, wq, D);
-  if (a->k_norm_w) widen_head(a->k_norm_w, wk, D);
+  if (a->q_norm_w) norm_weights(a->q_norm_w, a->norm_style == 1, wq);
+  if (a->k_norm_w) norm_weights(a->k_norm_w, a->norm_style == 1, wk);
 
   for (int32_t b = 0; b < a->B; ++b) {
     int64_t lo = a->q_indptr[b], hi = a->q_indptr[b + 1], L = a->seq_lens[b];
@@ -204,7 +220,7 @@ int fqro_append_paged(const fqro_append_args* a) {
        * r + L - q_indptr[b + 1]; the KV slot always uses that position. */
       int64_t p_slot = r + L - hi;
       int64_t pos = a->positions ? a->positions[r] : p_slot;
-      int64_t page = a->page_table[(int64_t)b * a->max_pages + p_slot / P];
+      int64_t page = paged ? a->page_table[(int64_t)b * a->max_pages + p_slot / P] : 0;
       int64_t row = p_slot % P;
       const float* cs = a->cos_sin + pos * a->rot_dim;
       const uint16_t* src = a->qkv + r * a->row_stride;
@@ -226,7 +242,12 @@ int fqro_append_paged(const fqro_append_args* a) {
           float amax = 0.0f;
           for (int i = 0; i < D; ++i) amax = fmaxf(amax, fabsf(y[i]));
           float qs = fmaxf(amax, 1e-6f) / a->upper_max;
-          a->q_scale[r * a->Hq + h] = qs;
+          /* decode layout [T, Hq]; prefill layout [B, Hq, ld] addressed by
+           * the token's index inside its request ([FI] "Contract") */
+          if (msl > 0)
+            a->q_scale[((int64_t)b * a->Hq + h) * ld + (r - lo)] = qs;
+          else
+            a->q_scale[r * a->Hq + h] = qs;
           uint8_t* q = (uint8_t*)a->out_q + o;
           for (int i = 0; i < D; ++i) q[i] = fqro_f32_to_e4m3_rn_satfinite(y[i] / qs);
         } else {
@@ -236,9 +257,14 @@ int fqro_append_paged(const fqro_append_args* a) {
             q[i] = fqro_f32_to_e4m3_rn_satfinite(y[i] * a->q_scale_inv);
         }
       }
+      void* kdst = paged ? a->k_cache : a->out_k;
+      void* vdst = paged ? a->v_cache : a->out_v;
       for (int kh = 0; kh < a->Hkv; ++kh) {
-        int64_t ko = page * a->k_page_stride + (row * a->Hkv + kh) * D;
-        int64_t vo = page * a->v_page_stride + (row * a->Hkv + kh) * D;
+        /* the cache slot, or row r of the caller-owned K / V outputs */
+        int64_t ko = paged ? page * a->k_page_stride + (row * a->Hkv + kh) * D
+                           : (r * a->Hkv + kh) * D;
+        int64_t vo = paged ? page * a->v_page_stride + (row * a->Hkv + kh) * D
+                           : (r * a->Hkv + kh) * D;
         /* K head */
         widen_head(src + (int64_t)(a->Hq + kh) * D, x, D);
         if (a->k_norm_w)
@@ -247,18 +273,18 @@ int fqro_append_paged(const fqro_append_args* a) {
           memcpy(y, x, sizeof y);
         rope(y, cs, a->rot_dim, a->rope_style);
         if (!fp8) {
-          uint16_t* k = (uint16_t*)a->k_cache + ko;
+          uint16_t* k = (uint16_t*)kdst + ko;
           for (int i = 0; i < D; ++i) k[i] = fqro_f32_to_bf16_rne(y[i]);
         } else {
-          uint8_t* k = (uint8_t*)a->k_cache + ko;
+          uint8_t* k = (uint8_t*)kdst + ko;
           for (int i = 0; i < D; ++i) k[i] = fqro_f32_to_e4m3_rn_satfinite(y[i] / a->k_scale);
         }
         /* V head: a bit copy in BF16, x / v_scale in FP8 */
         const uint16_t* vs = src + (int64_t)(a->Hq + a->Hkv + kh) * D;
         if (!fp8) {
-          memcpy((uint16_t*)a->v_cache + vo, vs, D * sizeof(uint16_t));
+          memcpy((uint16_t*)vdst + vo, vs, D * sizeof(uint16_t));
         } else {
-          uint8_t* v = (uint8_t*)a->v_cache + vo;
+          uint8_t* v = (uint8_t*)vdst + vo;
           for (int i = 0; i < D; ++i)
             v[i] = fqro_f32_to_e4m3_rn_satfinite(fqro_bf16_to_f32(vs[i]) / a->v_scale);
         }
@@ -267,9 +293,10 @@ int fqro_append_paged(const fqro_append_args* a) {
   }
 
   /* Rows [last + 1, page_size) of every request's last page are zeroed in
-   * both caches ([FI] "Contract"); a request with L == 0 has no last page. */
+   * both caches ([FI] "Contract"); a request with L == 0 has no last page.
+   * Redirected K/V writes leave the caches alone ([FI] review). */
   const int64_t esize = fp8 ? 1 : 2;
-  for (int32_t b = 0; b < a->B; ++b) {
+  for (int32_t b = 0; paged && b < a->B; ++b) {
     int64_t L = a->seq_lens[b];
     if (L <= 0) continue;
     int64_t last = (L - 1) % P;
@@ -291,7 +318,7 @@ int fqro_append_paged(const fqro_append_args* a) {
 /* ------------------------------------------------------------------------ */
 int fqro_concat_mla_cache(const fqro_mla_args* a) {
   if (fqro_validate(a->q_indptr, a->seq_lens, a->B, a->T, a->max_blocks,
-                    a->block_size, a->cos_sin_rows, a->positions)) {
+                    a->block_size, a->cos_sin_rows, a->positions, 0, 1)) {
     for (int32_t b = 0; b < a->B; ++b) a->flags[b] = -1;
     return 1;
   }

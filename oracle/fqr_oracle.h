@@ -46,10 +46,13 @@ void fqro_rope_neox(float* y, const float* cs_row, int rot);
 void fqro_rope_gptj(float* y, const float* cs_row, int rot);
 
 /* ---- metadata validation ------------------------------------------------ */
-/* Returns 1 if the batch metadata is malformed (any request), else 0. */
+/* Returns 1 if the batch metadata is malformed (any request), else 0.
+ * paged = 0 skips the page-overrun check (no page is addressed);
+ * max_seqlen > 0 adds n_b <= max_seqlen. */
 int fqro_validate(const int32_t* q_indptr, const int32_t* seq_lens, int32_t B,
                   int32_t T, int32_t max_pages, int32_t page_size,
-                  int32_t cos_sin_rows, const int64_t* positions);
+                  int32_t cos_sin_rows, const int64_t* positions,
+                  int32_t max_seqlen, int32_t paged);
 
 /* ---- the paged append --------------------------------------------------- */
 typedef struct {
@@ -76,8 +79,14 @@ typedef struct {
   void* v_cache;
   int64_t k_page_stride, v_page_stride;   /* elements between pages         */
   void* out_q;                /* [T, Hq, 128] bf16 bits or e4m3 codes        */
-  float* q_scale;             /* [T, Hq] (policy 1) or NULL                  */
+  float* q_scale;             /* policy 1: [T, Hq] (max_seqlen 0) or
+                                 [B, Hq, round_up(max_seqlen, 128)]; else NULL */
   int32_t* flags;             /* [B]                                         */
+  int32_t max_seqlen;         /* policy 1: 0 decode layout, > 0 prefill layout
+                                 and the n_b <= max_seqlen check              */
+  int32_t norm_style;         /* 0: y = x_hat * w, 1 (Gemma): x_hat * (1 + w) */
+  void* out_k;                /* [T, Hkv, 128] or NULL (paged caches)        */
+  void* out_v;
 } fqro_append_args;
 
 /* Returns 0 after a valid call, 1 when the metadata was flagged. */

@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libfqr.so")
 FQR_OK, FQR_EINVAL, FQR_ENOTSUP, FQR_ECUDA = 0, 1, 2, 3
 SCHEDULE_AUTO, SCHEDULE_LATENCY, SCHEDULE_STREAMING = 0, 1, 2
 FLAG_TIMEOUT = -2
+NORM_RMS, NORM_GEMMA = 0, 1
 HEAD_DIM = 128
 MAX_BATCH = 16384
 
@@ -43,6 +44,7 @@ class AppendParams(ctypes.Structure):
         ("quant_policy", c_i32),
         ("q_scale_inv", c_vp), ("k_scale", c_vp), ("v_scale", c_vp), ("upper_max", c_f32),
         ("out_q", c_vp), ("q_scale", c_vp), ("flags", c_vp), ("schedule", c_i32),
+        ("max_seqlen", c_i32), ("norm_style", c_i32), ("out_k", c_vp), ("out_v", c_vp),
     ]
 
 
@@ -114,25 +116,34 @@ def append_params(qkv, cos_sin_cache, q_indptr, seq_lens, page_table, k_cache, v
                   positions=None, rope_style: int = 0, rot_dim: Optional[int] = None,
                   quant_policy: int = 0, q_scale=None, q_scale_inv=None, k_scale=None,
                   v_scale=None, upper_max: float = 448.0,
-                  schedule: int = SCHEDULE_AUTO) -> AppendParams:
-    """Fill an AppendParams from tensors (shapes as in include/fqr.h)."""
+                  schedule: int = SCHEDULE_AUTO, max_seqlen: int = 0,
+                  norm_style: int = NORM_RMS, out_k=None, out_v=None) -> AppendParams:
+    """Fill an AppendParams from tensors (shapes as in include/fqr.h).  With
+    out_k / out_v ([T, Hkv, 128]) the K/V payloads go there; k_cache, v_cache
+    and page_table may then be None."""
     T = int(qkv.shape[0])
+    kv = k_cache if k_cache is not None else out_k
+    paged = k_cache is not None
     return AppendParams(
         qkv=_ptr(qkv), qkv_row_stride=int(qkv.stride(0)) if T > 0 else int(qkv.shape[1]),
-        T=T, B=int(seq_lens.numel()), Hq=int(out_q.shape[1]), Hkv=int(k_cache.shape[2]),
-        head_dim=int(k_cache.shape[3]),
+        T=T, B=int(seq_lens.numel()), Hq=int(out_q.shape[1]), Hkv=int(kv.shape[-2]),
+        head_dim=int(kv.shape[-1]),
         q_norm_w=_ptr(q_norm_w), k_norm_w=_ptr(k_norm_w), eps=float(eps),
         cos_sin_cache=_ptr(cos_sin_cache), cos_sin_rows=int(cos_sin_cache.shape[0]),
         rot_dim=int(cos_sin_cache.shape[1] if rot_dim is None else rot_dim),
         rope_style=int(rope_style), positions=_ptr(positions),
         q_indptr=_ptr(q_indptr), seq_lens=_ptr(seq_lens), page_table=_ptr(page_table),
-        max_pages=int(page_table.shape[1]),
-        k_cache=_ptr(k_cache), v_cache=_ptr(v_cache), num_pages=int(k_cache.shape[0]),
-        page_size=int(k_cache.shape[1]),
-        k_page_stride=int(k_cache.stride(0)), v_page_stride=int(v_cache.stride(0)),
+        max_pages=int(page_table.shape[1]) if page_table is not None else 0,
+        k_cache=_ptr(k_cache), v_cache=_ptr(v_cache),
+        num_pages=int(k_cache.shape[0]) if paged else 0,
+        page_size=int(k_cache.shape[1]) if paged else 0,
+        k_page_stride=int(k_cache.stride(0)) if paged else 0,
+        v_page_stride=int(v_cache.stride(0)) if paged else 0,
         quant_policy=int(quant_policy), q_scale_inv=_ptr(q_scale_inv),
         k_scale=_ptr(k_scale), v_scale=_ptr(v_scale), upper_max=float(upper_max),
-        out_q=_ptr(out_q), q_scale=_ptr(q_scale), flags=_ptr(flags), schedule=int(schedule))
+        out_q=_ptr(out_q), q_scale=_ptr(q_scale), flags=_ptr(flags), schedule=int(schedule),
+        max_seqlen=int(max_seqlen), norm_style=int(norm_style),
+        out_k=_ptr(out_k), out_v=_ptr(out_v))
 
 
 def append_paged(qkv, cos_sin_cache, q_indptr, seq_lens, page_table, k_cache, v_cache,
@@ -147,7 +158,7 @@ def append_paged(qkv, cos_sin_cache, q_indptr, seq_lens, page_table, k_cache, v_
     Raises FqrError on a host-side argument error."""
     p = append_params(qkv, cos_sin_cache, q_indptr, seq_lens, page_table, k_cache, v_cache,
                       out_q, flags, **kw)
-    rc = append_paged_raw(p, _stream(stream, k_cache.device))
+    rc = append_paged_raw(p, _stream(stream, qkv.device))
     if rc != FQR_OK:
         raise FqrError(rc)
 
@@ -214,4 +225,5 @@ __all__ = ["LIB", "LIB_PATH", "AppendParams", "MlaParams", "FqrError", "strerror
            "append_params", "append_paged", "append_paged_raw", "mla_params",
            "concat_mla_cache", "concat_mla_cache_raw", "FQR_OK", "FQR_EINVAL",
            "FQR_ENOTSUP", "FQR_ECUDA", "HEAD_DIM", "MAX_BATCH", "SCHEDULE_AUTO",
-           "SCHEDULE_LATENCY", "SCHEDULE_STREAMING", "FLAG_TIMEOUT"]
+           "SCHEDULE_LATENCY", "SCHEDULE_STREAMING", "FLAG_TIMEOUT", "NORM_RMS",
+           "NORM_GEMMA"]

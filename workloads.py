@@ -78,6 +78,10 @@ class AppendWorkload:
     k_scale: float = 1.0
     v_scale: float = 1.0
     upper_max: float = 448.0
+    max_seqlen: int = 0        # policy 1: > 0 selects the prefill q_scale layout
+    norm_style: int = 0        # 0: x_hat * w, 1 (Gemma): x_hat * (1 + w)
+    out_kv: bool = False       # K/V to caller-owned [T, Hkv, 128] buffers
+    gate_heads: int = 0        # G heads after V in each row (never read)
     extra: dict = field(default_factory=dict)
 
     @property
@@ -91,6 +95,14 @@ class AppendWorkload:
     @property
     def kv_esize(self) -> int:
         return 2 if self.quant_policy == 0 else 1
+
+    @property
+    def q_scale_shape(self) -> tuple:
+        """Decode layout [T, Hq]; with max_seqlen > 0 the prefill layout
+        [B, Hq, round_up(max_seqlen, 128)]."""
+        if self.max_seqlen > 0:
+            return (self.B, self.Hq, -(-self.max_seqlen // 128) * 128)
+        return (self.T, self.Hq)
 
     @property
     def q_esize(self) -> int:
@@ -142,11 +154,13 @@ def make_append(*, name="custom", seed=0, n_new, seq_lens, Hq, Hkv, page_size,
                 norm=True, rot_dim=HEAD_DIM, rope_style=0, theta=1e6,
                 cos_sin_rows=None, row_pad=0, positions=None,
                 q_scale_inv=1.0, k_scale=1.0, v_scale=1.0, upper_max=448.0,
-                eps=1e-6) -> AppendWorkload:
+                eps=1e-6, max_seqlen=0, norm_style=0, out_kv=False,
+                gate_heads=0) -> AppendWorkload:
     """Build a paged-append workload from per-request new-token counts and
     post-append lengths.  The page table is a seeded random permutation of
     `num_pages` page ids reshaped to [B, max_pages] (num_pages defaults to
-    B * max_pages)."""
+    B * max_pages).  `gate_heads` appends that many 128-wide G heads to every
+    row ([Q | K | V | G]), ahead of any `row_pad`."""
     rng = rng_for(seed)
     n_new = np.asarray(n_new, dtype=np.int64)
     seq_lens = np.asarray(seq_lens, dtype=np.int32)
@@ -155,7 +169,7 @@ def make_append(*, name="custom", seed=0, n_new, seq_lens, Hq, Hkv, page_size,
     q_indptr = np.zeros(B + 1, dtype=np.int32)
     q_indptr[1:] = np.cumsum(n_new)
     H = Hq + 2 * Hkv
-    row_stride = H * HEAD_DIM + row_pad
+    row_stride = (H + gate_heads) * HEAD_DIM + row_pad
     qkv = bf16_normal(rng, (T, row_stride), sigma=qkv_sigma)
     qw = bf16_normal(rng, (HEAD_DIM,), mean=1.0, sigma=0.1) if norm else None
     kw = bf16_normal(rng, (HEAD_DIM,), mean=1.0, sigma=0.1) if norm else None
@@ -178,7 +192,8 @@ def make_append(*, name="custom", seed=0, n_new, seq_lens, Hq, Hkv, page_size,
         q_indptr=q_indptr, seq_lens=seq_lens, page_table=page_table,
         num_pages=num_pages, page_size=page_size, quant_policy=quant_policy,
         q_scale_inv=q_scale_inv, k_scale=k_scale, v_scale=v_scale,
-        upper_max=upper_max)
+        upper_max=upper_max, max_seqlen=max_seqlen, norm_style=norm_style,
+        out_kv=out_kv, gate_heads=gate_heads)
 
 
 def tiny_decode_bf16(seed=1001) -> AppendWorkload:
@@ -294,11 +309,51 @@ def make_mla(*, seed=0, n_new, seq_lens, Hq, block_size, max_blocks,
                        cache_fp8=cache_fp8, kv_scale=kv_scale)
 
 
+def prefill_dynq_gemma(seed=1006, q_len=129) -> AppendWorkload:
+    """Dynamic-Q prefill with the [B, Hq, round_up(max_seqlen, 128)] q_scale
+    layout and the Gemma-style norm: 4 requests x q_len new tokens each,
+    max_seqlen = q_len (the pages' padding-edge rows use q_len 127 / 128 /
+    129), Hq 64 / Hkv 8, page 64, prior context U[0, 1024], k/v scale 0.05."""
+    rng = rng_for(seed + 7)
+    prior = rng.integers(0, 1024, size=4, endpoint=True)
+    L = prior + q_len
+    return make_append(name=f"prefill_dynq_gemma_B4_q{q_len}_h64x8_p64", seed=seed,
+                       n_new=[q_len] * 4, seq_lens=L, Hq=64, Hkv=8, page_size=64,
+                       max_pages=64, num_pages=4096, quant_policy=1,
+                       cos_sin_rows=2048, k_scale=0.05, v_scale=0.05,
+                       max_seqlen=q_len, norm_style=1)
+
+
+def decode_out_kv_bf16(seed=1007) -> AppendWorkload:
+    """Decode into caller-owned K/V buffers (no paged cache, no tail): 128
+    requests x 1 token, Hq 32 / Hkv 8, BF16."""
+    rng = rng_for(seed + 7)
+    L = rng.integers(1, 8192, size=128, endpoint=True)
+    return make_append(name="decode_out_kv_bf16_B128_h32x8", seed=seed,
+                       n_new=[1] * 128, seq_lens=L, Hq=32, Hkv=8, page_size=16,
+                       max_pages=512, num_pages=1, quant_policy=0,
+                       cos_sin_rows=8192, out_kv=True)
+
+
+def gate_tail_decode_bf16(seed=1008) -> AppendWorkload:
+    """Gated-attention rows [Q | K | V | G] (one G head per Q head, left
+    untouched): 128 requests x 1 token, Hq 32 / Hkv 4, page 16, BF16 cache."""
+    rng = rng_for(seed + 7)
+    L = rng.integers(1, 8192, size=128, endpoint=True)
+    return make_append(name="gate_tail_decode_bf16_B128_h32x4g32_p16", seed=seed,
+                       n_new=[1] * 128, seq_lens=L, Hq=32, Hkv=4, page_size=16,
+                       max_pages=512, num_pages=65536, quant_policy=0,
+                       cos_sin_rows=8192, gate_heads=32)
+
+
 APPEND_CONFIGS = {
     "tiny_decode_bf16": tiny_decode_bf16,
     "qwen3_decode_bf16": qwen3_decode_bf16,
     "fp8_decode_dynamic": fp8_decode_dynamic,
     "ragged_prefill_fp8": ragged_prefill_fp8,
+    "prefill_dynq_gemma": prefill_dynq_gemma,
+    "decode_out_kv_bf16": decode_out_kv_bf16,
+    "gate_tail_decode_bf16": gate_tail_decode_bf16,
 }
 MLA_CONFIGS = {"mla_decode": mla_decode}
 
@@ -319,9 +374,10 @@ def append_bytes(w: AppendWorkload) -> dict:
     reads += (2 * D * 2) if w.q_norm_w is not None else 0
     reads += T * w.rot_dim * 4
     reads += 4 * (B + 1) + 4 * B
-    # one page-table entry per distinct (request, page) touched
+    # one page-table entry per distinct (request, page) touched (none when
+    # K/V go to caller-owned buffers)
     touched = 0
-    for b in range(B):
+    for b in range(B if not w.out_kv else 0):
         lo, hi, L = int(w.q_indptr[b]), int(w.q_indptr[b + 1]), int(w.seq_lens[b])
         pages = set()
         for r in range(lo, hi):
@@ -335,7 +391,7 @@ def append_bytes(w: AppendWorkload) -> dict:
     bq, bkv = w.q_esize, w.kv_esize
     writes = T * Hq * D * bq + T * 2 * Hkv * D * bkv
     tail_rows = 0
-    for b in range(B):
+    for b in range(B if not w.out_kv else 0):   # no tail without paged caches
         L = int(w.seq_lens[b])
         if L > 0:
             tail_rows += P - 1 - (L - 1) % P
