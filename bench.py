@@ -226,9 +226,13 @@ class AppendBench:
                       seq_lens=self._d(w.seq_lens), page_table=self._d(w.page_table),
                       out_q=torch.empty((w.T, w.Hq, 128), dtype=dt if w.quant_policy == 0
                                         else torch.uint8, device=device),
-                      q_scale=torch.empty((max(w.T, 1), w.Hq), dtype=torch.float32,
-                                          device=device),
+                      q_scale=torch.empty(w.q_scale_shape if w.T else (1, w.Hq),
+                                          dtype=torch.float32, device=device),
                       flags=torch.empty((w.B,), dtype=torch.int32, device=device))
+            if w.out_kv:   # caller-owned K/V rows instead of the paged caches
+                kdt = dt if w.quant_policy == 0 else torch.uint8
+                st["out_k"] = torch.empty((w.T, w.Hkv, 128), dtype=kdt, device=device)
+                st["out_v"] = torch.empty((w.T, w.Hkv, 128), dtype=kdt, device=device)
             st["params"] = self._params(w, st)
             self.reps.append(st)
 
@@ -247,7 +251,8 @@ class AppendBench:
                     q_scale_inv=self.scales["q_scale_inv"] if w.quant_policy == 2 else None,
                     k_scale=self.scales["k_scale"] if w.quant_policy else None,
                     v_scale=self.scales["v_scale"] if w.quant_policy else None,
-                    upper_max=w.upper_max, schedule=self.schedule)
+                    upper_max=w.upper_max, schedule=self.schedule, max_seqlen=w.max_seqlen,
+                    norm_style=w.norm_style, out_k=st.get("out_k"), out_v=st.get("out_v"))
 
     def _params(self, w, st):
         return self.fqr.append_params(st["qkv"], self.cs, st["q_indptr"], st["seq_lens"],

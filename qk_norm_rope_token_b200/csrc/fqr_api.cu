@@ -28,24 +28,39 @@ int check_append(const fqr_append_params* p) {
   if (p->quant_policy == 1 &&
       !(std::isfinite(p->upper_max) && p->upper_max > 0.0f && p->upper_max <= 448.0f))
     return FQR_EINVAL;
-  if (p->page_size <= 0 || p->num_pages <= 0 || p->max_pages <= 0 || p->cos_sin_rows <= 0)
+  if (p->cos_sin_rows <= 0) return FQR_EINVAL;
+  // caller-owned K/V rows (both or neither) replace the paged caches
+  const bool owned = p->out_k != nullptr || p->out_v != nullptr;
+  if (owned && (!p->out_k || !p->out_v || !aligned(p->out_k, 16) || !aligned(p->out_v, 16)))
     return FQR_EINVAL;
-  // tail rows of the whole batch are counted in 32 bits
-  if (2 * static_cast<int64_t>(p->B) * (p->page_size - 1) >= (int64_t{1} << 31)) return FQR_EINVAL;
   const int64_t H = static_cast<int64_t>(p->Hq) + 2 * static_cast<int64_t>(p->Hkv);
   if (p->qkv_row_stride < H * FQR_HEAD_DIM || p->qkv_row_stride % 8 != 0) return FQR_EINVAL;
   const int64_t esize = p->quant_policy == 0 ? 2 : 1;
-  const int64_t page_elems = static_cast<int64_t>(p->page_size) * p->Hkv * FQR_HEAD_DIM;
-  if (p->k_page_stride < page_elems || p->v_page_stride < page_elems) return FQR_EINVAL;
-  if ((p->k_page_stride * esize) % 16 != 0 || (p->v_page_stride * esize) % 16 != 0)
-    return FQR_EINVAL;
+  if (!owned) {
+    if (p->page_size <= 0 || p->num_pages <= 0 || p->max_pages <= 0) return FQR_EINVAL;
+    // tail rows of the whole batch are counted in 32 bits
+    if (2 * static_cast<int64_t>(p->B) * (p->page_size - 1) >= (int64_t{1} << 31))
+      return FQR_EINVAL;
+    const int64_t page_elems = static_cast<int64_t>(p->page_size) * p->Hkv * FQR_HEAD_DIM;
+    if (p->k_page_stride < page_elems || p->v_page_stride < page_elems) return FQR_EINVAL;
+    if ((p->k_page_stride * esize) % 16 != 0 || (p->v_page_stride * esize) % 16 != 0)
+      return FQR_EINVAL;
+    if (!p->page_table || !p->k_cache || !p->v_cache) return FQR_EINVAL;
+    if (!aligned(p->k_cache, 16) || !aligned(p->v_cache, 16) || !aligned(p->page_table, 4))
+      return FQR_EINVAL;
+  }
+  // the dynamic-Q prefill layout [B, Hq, round_up(max_seqlen, 128)] is indexed in 32 bits
+  if (p->max_seqlen < 0) return FQR_EINVAL;
+  if (p->quant_policy == 1 && p->max_seqlen > 0 &&
+      static_cast<int64_t>(p->B) * p->Hq * ((static_cast<int64_t>(p->max_seqlen) + 127) / 128 * 128) >=
+          (int64_t{1} << 31))
+    return FQR_ENOTSUP;
+  if (p->norm_style != FQR_NORM_RMS && p->norm_style != FQR_NORM_GEMMA) return FQR_EINVAL;
   // required pointers and their alignment
-  if (!p->q_indptr || !p->seq_lens || !p->page_table || !p->flags) return FQR_EINVAL;
-  if (!p->k_cache || !p->v_cache || !p->cos_sin_cache) return FQR_EINVAL;
-  if (!aligned(p->k_cache, 16) || !aligned(p->v_cache, 16) || !aligned(p->cos_sin_cache, 16))
-    return FQR_EINVAL;
-  if (!aligned(p->q_indptr, 4) || !aligned(p->seq_lens, 4) || !aligned(p->page_table, 4) ||
-      !aligned(p->flags, 4) || !aligned(p->positions, 8))
+  if (!p->q_indptr || !p->seq_lens || !p->flags || !p->cos_sin_cache) return FQR_EINVAL;
+  if (!aligned(p->cos_sin_cache, 16)) return FQR_EINVAL;
+  if (!aligned(p->q_indptr, 4) || !aligned(p->seq_lens, 4) || !aligned(p->flags, 4) ||
+      !aligned(p->positions, 8))
     return FQR_EINVAL;
   if (p->T > 0) {
     if (!p->qkv || !p->out_q || !aligned(p->qkv, 16) || !aligned(p->out_q, 16))

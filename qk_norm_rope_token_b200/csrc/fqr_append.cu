@@ -16,10 +16,14 @@ namespace fqr {
 int launch_append(const fqr_append_params& p, cudaStream_t stream) {
   HeadParams hp;
   const int es = p.quant_policy == 0 ? 2 : 1;
-  hp.pdiv = FastDiv(static_cast<uint32_t>(p.page_size));
+  const bool owned = p.out_k != nullptr;
+  // with caller-owned K/V no page is addressed: a page size of 1 keeps the
+  // slot arithmetic defined (its results are not used)
+  const int page_size = owned ? 1 : p.page_size;
+  hp.pdiv = FastDiv(static_cast<uint32_t>(page_size));
   hp.Hq = p.Hq;
   hp.Hkv = p.Hkv;
-  hp.page_size = p.page_size;
+  hp.page_size = page_size;
   hp.row_bytes = p.Hkv * kHeadDim * es;
   hp.rot = p.rot_dim;
   hp.has_qw = p.q_norm_w != nullptr;
@@ -35,6 +39,11 @@ int launch_append(const fqr_append_params& p, cudaStream_t stream) {
   hp.v_scale = p.v_scale;
   hp.out_q = p.out_q;
   hp.q_scale = p.q_scale;
+  hp.gemma = p.norm_style == FQR_NORM_GEMMA;
+  hp.qs_prefill = p.quant_policy == 1 && p.max_seqlen > 0;
+  hp.qs_ld = hp.qs_prefill ? (p.max_seqlen + 127) / 128 * 128 : 1;
+  hp.out_k = static_cast<char*>(p.out_k);
+  hp.out_v = static_cast<char*>(p.out_v);
 
   int schedule = p.schedule;
   if (schedule == FQR_SCHEDULE_AUTO) {

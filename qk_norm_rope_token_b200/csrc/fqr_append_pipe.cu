@@ -14,7 +14,7 @@
 //     validation prologue.  The producer's 32 lanes resolve request, position
 //     and page id of 32 units in parallel; the cos/sin copy is issued before
 //     the page id is known, and the stage header (slot, page, position, last
-//     row) is published by the arrive that completes the phase.
+//     row, q_scale index) is published by the arrive that completes the phase.
 //   * consumer warps take 4 heads at a time from the stage (fqr_head.cuh),
 //     store straight to out_q / the cache slot and release the stage on its
 //     "empty" mbarrier; the quad -> warp assignment rotates every unit.
@@ -32,11 +32,13 @@ constexpr int kConsumers = 8;
 constexpr int kPipeThreads = (kConsumers + 1) * 32;
 constexpr int kMaxStages = 8;
 constexpr int kFixedSmem = 1280;  // barriers (128) + fp32 weights (1024) + spare
+constexpr int kHeader = 32;       // stage header bytes (keeps the copies 16-byte aligned)
 
 // Stage header, written by the producer before it arrives on "full".
 struct StageInfo {
-  int slot_row, page, pos, is_last;
+  int slot_row, page, pos, is_last, qs;
 };
+static_assert(sizeof(StageInfo) <= kHeader, "stage header");
 
 struct PipeArgs {
   HeadParams hp;
@@ -55,6 +57,8 @@ struct PipeArgs {
   const int32_t* seq_lens;
   const int32_t* page_table;
   int max_pages;
+  int64_t slot_cap;  // max_pages * page_size; INT64_MAX with caller-owned K/V
+  int max_seqlen;    // > 0: the dynamic-Q prefill check n_b <= max_seqlen
   int32_t* flags;
   int stages, stage_bytes;
 };
@@ -89,7 +93,7 @@ __device__ __forceinline__ void issue_heads(const PipeArgs& a, unsigned char* st
   unit_heads(a, u, t, h0, nh);
   const uint32_t bytes = static_cast<uint32_t>(nh) * kHeadDim * 2;
   mbar_expect_tx(bar, bytes);
-  bulk_g2s(st + 16 + a.cs_bytes,
+  bulk_g2s(st + kHeader + a.cs_bytes,
            a.qkv + static_cast<int64_t>(t) * a.row_stride + static_cast<int64_t>(h0) * kHeadDim,
            bytes, bar);
 }
@@ -106,7 +110,7 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
   uint32_t eph = 1;  // parity of the empty-phase to wait for (previous use of stage s)
   for (int i0 = 0; i0 < nunits && ok; i0 += 32) {
     // lane j prepares unit i0 + j in parallel with the others
-    StageInfo info{0, 0, 0, 0};  // slot_row, page, pos, is_last
+    StageInfo info{0, 0, 0, 0, 0};  // slot_row, page, pos, is_last, qs
     int need_cs = 0;
     if (i0 + lane < nunits) {
       int t, h0, nh;
@@ -118,7 +122,9 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
       info.slot_row = p - pidx * a.hp.page_size;
       info.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : p;
       info.is_last = t == end - 1;
-      if (h0 + nh > a.hp.Hq)  // the unit holds K or V heads: it needs the page id
+      info.qs = q_scale_row(a.hp, t, b, t - s_indptr[b]);
+      // a unit with K or V heads needs the page id (unless K/V go to owned rows)
+      if (h0 + nh > a.hp.Hq && a.hp.out_k == nullptr)
         info.page = __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx);
       need_cs = (h0 < a.hp.Hq + a.hp.Hkv) && a.cs_bulk;
     }
@@ -141,7 +147,7 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
           if (csj) {
             const uint32_t cb = static_cast<uint32_t>(a.hp.rot) * 4;
             mbar_expect_tx(fb, cb);
-            bulk_g2s(st + 16, a.cs + static_cast<int64_t>(posj) * a.hp.rot, cb, fb);
+            bulk_g2s(st + kHeader, a.cs + static_cast<int64_t>(posj) * a.hp.rot, cb, fb);
           }
         }
       }
@@ -149,7 +155,8 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
       if (!ok) break;
       const StageInfo sj{__shfl_sync(0xffffffffu, info.slot_row, j),
                          __shfl_sync(0xffffffffu, info.page, j), posj,
-                         __shfl_sync(0xffffffffu, info.is_last, j)};
+                         __shfl_sync(0xffffffffu, info.is_last, j),
+                         __shfl_sync(0xffffffffu, info.qs, j)};
       if (lane == 0) {
         *reinterpret_cast<StageInfo*>(st) = sj;
         mbar_arrive(fb);  // release: the header is visible once the phase completes
@@ -193,8 +200,8 @@ __device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t
     }
     const unsigned char* st = stages + static_cast<size_t>(s) * a.stage_bytes;
     const StageInfo info = *reinterpret_cast<const StageInfo*>(st);
-    const RowCtx r{t, info.slot_row, info.pos, info.page, info.is_last};
-    const float* cs_row = CSB ? reinterpret_cast<const float*>(st + 16)
+    const RowCtx r{t, info.slot_row, info.pos, info.page, info.is_last, info.qs};
+    const float* cs_row = CSB ? reinterpret_cast<const float*>(st + kHeader)
                               : a.cs + static_cast<int64_t>(info.pos) * a.hp.rot;
     const int h0 = c * a.chunk_heads, nh = min(a.H - h0, a.chunk_heads);
     const int nq = (nh + 3) >> 2;
@@ -204,7 +211,7 @@ __device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t
       const int hl = 4 * q + g;
       uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = xa;
       if (hl < nh) {
-        const unsigned char* src = st + 16 + a.cs_bytes + hl * (kHeadDim * 2) + 16 * l8;
+        const unsigned char* src = st + kHeader + a.cs_bytes + hl * (kHeadDim * 2) + 16 * l8;
         xa = ld_smem_v4(src);
         xb = ld_smem_v4(src + 128);
       }
@@ -229,6 +236,7 @@ __device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t
 // consumer warp of the grid.
 template <int POLICY>
 __device__ void zero_empty_request_tails(const PipeArgs& a, const int* s_indptr, const int* s_seq) {
+  if (a.hp.out_k != nullptr) return;  // caller-owned K/V: the caches are not touched
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int W = gridDim.x * kConsumers;
   for (int b = blockIdx.x * kConsumers + warp; b < a.B; b += W) {
@@ -279,10 +287,10 @@ __global__ void __launch_bounds__(kPipeThreads, 2) pipe_append_kernel(const Pipe
       issue_heads(a, stages + static_cast<size_t>(i) * a.stage_bytes, u0 + i, &full[i]);
   }
   const MetaRegs meta = meta_prefetch(a.q_indptr, a.seq_lens, a.B);
-  weight_store(s_w, weight_prefetch(a.qw, a.kw));
+  weight_store(s_w, weight_prefetch(a.qw, a.kw, a.hp.gemma));
 
-  const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
-               static_cast<int64_t>(a.max_pages) * a.hp.page_size, a.cs_rows};
+  const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T,
+               a.B,         a.slot_cap,  a.cs_rows,  a.max_seqlen};
   if (stage_and_validate(m, s_indptr, s_seq, meta)) {
     if (producer && lane == 0) {  // drain the copies issued before the verdict
       for (int i = 0; i < pre; ++i) {
@@ -340,6 +348,8 @@ int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStr
   a.seq_lens = p.seq_lens;
   a.page_table = p.page_table;
   a.max_pages = p.max_pages;
+  a.slot_cap = hp.out_k != nullptr ? INT64_MAX : static_cast<int64_t>(p.max_pages) * p.page_size;
+  a.max_seqlen = p.quant_policy == 1 ? p.max_seqlen : 0;
   a.flags = p.flags;
 
   int dev = 0, sms = 0, smem_optin = 0, smem_sm = 0;
@@ -352,7 +362,7 @@ int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStr
     return FQR_ECUDA;
 
   const int64_t meta = static_cast<int64_t>(2 * p.B + 1) * sizeof(int);
-  auto stage_bytes = [&](int hc) { return 16 + a.cs_bytes + hc * kHeadDim * 2; };
+  auto stage_bytes = [&](int hc) { return kHeader + a.cs_bytes + hc * kHeadDim * 2; };
   // a row that does not fit two stages beside the metadata is split into
   // chunks of whole quads
   int hc = a.H;

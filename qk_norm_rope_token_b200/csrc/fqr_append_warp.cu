@@ -38,6 +38,8 @@ struct WarpArgs {
   const int32_t* seq_lens;
   const int32_t* page_table;
   int max_pages;
+  int64_t slot_cap;  // max_pages * page_size; INT64_MAX with caller-owned K/V
+  int max_seqlen;    // > 0: the dynamic-Q prefill check n_b <= max_seqlen
   int32_t* flags;
 };
 
@@ -76,7 +78,8 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   // heads and its own request's metadata (request guessed as b = t: one new
   // row per request, the decode case).
   const MetaRegs meta = meta_prefetch(a.q_indptr, a.seq_lens, a.B);
-  const float wreg = weight_prefetch(a.qw, a.kw);
+  const float wreg = weight_prefetch(a.qw, a.kw, a.hp.gemma);
+  const bool paged = a.hp.out_k == nullptr;
   uint4 pa = make_uint4(0u, 0u, 0u, 0u), pb = pa;
   const bool head0 = gwarp < a.n_head;
   int t0 = 0, h0 = a.H, gb = 0, e_lo = 0, e_hi = 0, e_L = 0;
@@ -94,20 +97,21 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   // ---- second round trip, started before the validation prologue when the
   // row's own metadata is consistent and every address it yields is in
   // bounds (the prologue still decides whether anything is written).
-  RowCtx r0{t0, 0, 0, 0, 0};
+  RowCtx r0{t0, 0, 0, 0, 0, 0};
   float2 c0[4], s0[4];
   bool early = false;
   if (head0 && h0 < a.H && e_lo <= t0 && t0 < e_hi) {
     const int p = t0 + e_L - e_hi;
     const int64_t pos = a.positions != nullptr ? e_pos : static_cast<int64_t>(p);
-    if (p >= 0 && p < static_cast<int64_t>(a.max_pages) * a.hp.page_size && pos >= 0 &&
-        pos < a.cs_rows) {
+    if (p >= 0 && p < a.slot_cap && pos >= 0 && pos < a.cs_rows) {
       early = true;
       const int pidx = static_cast<int>(a.hp.pdiv.div(static_cast<uint32_t>(p)));
       r0.slot_row = p - pidx * a.hp.page_size;
       r0.pos = static_cast<int>(pos);
       r0.is_last = t0 == e_hi - 1;
-      if (h0 >= a.hp.Hq || r0.is_last)  // K/V slot, or the tail share of the last row
+      r0.qs = q_scale_row(a.hp, t0, gb, t0 - e_lo);
+      // K/V slot, or the tail share of the last row
+      if (paged && (h0 >= a.hp.Hq || r0.is_last))
         r0.page = __ldg(a.page_table + static_cast<int64_t>(gb) * a.max_pages + pidx);
       if (h0 < a.hp.Hq + a.hp.Hkv)
         load_cs<STYLE, false>(a.cs + pos * a.hp.rot, a.hp.rot, l8, c0, s0);
@@ -115,8 +119,8 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   }
   weight_store(s_w, wreg);
 
-  const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
-               static_cast<int64_t>(a.max_pages) * a.hp.page_size, a.cs_rows};
+  const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T,
+               a.B,         a.slot_cap,  a.cs_rows,  a.max_seqlen};
   if (stage_and_validate(m, s_indptr, s_seq, meta)) return;
 
   const int n_tasks = a.n_head + a.B;
@@ -129,7 +133,7 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
       if (w == gwarp && early) {  // the batch is valid: the early lookups stand
         process_quad_cs<POLICY, STYLE, false>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, s_w, l8,
                                               gmask);
-        if (r0.is_last) zero_tail_share(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane);
+        if (paged && r0.is_last) zero_tail_share(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane);
         continue;
       }
       const int h = quad * 4 + g;
@@ -142,18 +146,19 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
       r.slot_row = p_slot - pidx * a.hp.page_size;
       r.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : p_slot;
       r.is_last = t == end - 1;
-      r.page = (h >= a.hp.Hq || r.is_last)
+      r.qs = q_scale_row(a.hp, t, b, t - s_indptr[b]);
+      r.page = paged && (h >= a.hp.Hq || r.is_last)
                    ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx)
                    : 0;
       // (a group past the last head only helps with the tail)
       const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
       process_quad<POLICY, STYLE, false, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, s_w, l8,
                                                 gmask);
-      if (r.is_last) zero_tail_share(a.hp, r.page, r.slot_row, quad, a.qdiv, lane);
+      if (paged && r.is_last) zero_tail_share(a.hp, r.page, r.slot_row, quad, a.qdiv, lane);
     } else {
       const int b = w - a.n_head;  // request task: tail of a request without new rows
       const int L = s_seq[b];
-      if (s_indptr[b] == s_indptr[b + 1] && L > 0)
+      if (paged && s_indptr[b] == s_indptr[b + 1] && L > 0)
         zero_request_tail<POLICY == 0 ? 2 : 1>(a.hp, a.page_table, a.max_pages, b, L, lane);
     }
   }
@@ -218,6 +223,8 @@ int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStr
   a.seq_lens = p.seq_lens;
   a.page_table = p.page_table;
   a.max_pages = p.max_pages;
+  a.slot_cap = hp.out_k != nullptr ? INT64_MAX : static_cast<int64_t>(p.max_pages) * p.page_size;
+  a.max_seqlen = p.quant_policy == 1 ? p.max_seqlen : 0;
   a.flags = p.flags;
   const size_t smem = warp_smem(p);
   WarpKernel k = select_warp(p.quant_policy, p.rope_style);

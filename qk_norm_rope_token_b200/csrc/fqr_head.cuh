@@ -29,7 +29,18 @@ struct HeadParams {
   const float* v_scale;
   void* out_q;
   float* q_scale;
+  int gemma;       // the norm scales by 1 + w (Gemma-style) instead of w
+  int qs_prefill;  // q_scale layout [B, Hq, qs_ld] (else [T, Hq])
+  int qs_ld;       // round_up(max_seqlen, 128) for the prefill layout
+  char* out_k;     // caller-owned K / V rows [T, Hkv, 128], or null: the paged caches
+  char* out_v;
 };
+
+// q_scale index of head 0 of packed row t, the i-th row of request b (the
+// head stride is 1 in the decode layout, qs_ld in the prefill layout).
+__device__ __forceinline__ int q_scale_row(const HeadParams& a, int t, int b, int i) {
+  return a.qs_prefill ? (b * a.Hq) * a.qs_ld + i : t * a.Hq;
+}
 
 // Where one packed row goes.
 struct RowCtx {
@@ -38,6 +49,7 @@ struct RowCtx {
   int pos;       // RoPE position
   int page;      // page id of the KV slot (valid when the row has K/V heads to store)
   int is_last;   // the row is its request's last: its K/V heads also zero the tail
+  int qs;        // q_scale index of head 0 (q_scale_row; dynamic Q only)
 };
 
 __device__ __forceinline__ float4 lds_f4(const float* p) {
@@ -75,12 +87,15 @@ __device__ __forceinline__ int weight_slot(int e) {
 // Stage both weight vectors (fp32, permuted) in s_w[0, 256); NULL -> ones.
 // For blocks of at least 256 threads: weight_prefetch loads one value per
 // thread at kernel entry, weight_store writes it after the first round trip.
-__device__ __forceinline__ float weight_prefetch(const uint16_t* qw, const uint16_t* kw) {
+// gemma: the Gemma-style norm scales by 1 + w (an fp32 add) instead of w.
+__device__ __forceinline__ float weight_prefetch(const uint16_t* qw, const uint16_t* kw,
+                                                 int gemma) {
   const int i = threadIdx.x;
   if (i >= 2 * kHeadDim) return 0.0f;
   const uint16_t* w = i < kHeadDim ? qw : kw;
-  return w != nullptr ? __uint_as_float(static_cast<uint32_t>(__ldg(w + (i & (kHeadDim - 1)))) << 16)
-                      : 1.0f;
+  if (w == nullptr) return 1.0f;  // (the norm is off for this tensor)
+  const float v = __uint_as_float(static_cast<uint32_t>(__ldg(w + (i & (kHeadDim - 1)))) << 16);
+  return gemma ? __fadd_rn(1.0f, v) : v;
 }
 __device__ __forceinline__ void weight_store(float* s_w, float v) {
   const int i = threadIdx.x;
@@ -259,7 +274,9 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
   if (is_v) {  // -------------------------------------------------------- V
     const int kh = h - a.Hq - a.Hkv;
     char* page_base = a.v_cache + static_cast<int64_t>(r.page) * a.v_page_bytes;
-    char* dst = page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
+    char* dst = a.out_v != nullptr
+                    ? a.out_v + (static_cast<int64_t>(r.t) * a.Hkv + kh) * kHeadDim * ES
+                    : page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
     if (POLICY == 0) {  // bit copy
       st_v4(dst + 16 * l8, xa);
       st_v4(dst + 128 + 16 * l8, xb);
@@ -267,7 +284,8 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
       divide_pairs(y, __ldg(a.v_scale));
       store_head<POLICY>(dst, y, l8);
     }
-    if (TAILS && r.is_last) zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
+    if (TAILS && r.is_last && a.out_v == nullptr)
+      zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
     return;
   }
 
@@ -329,7 +347,7 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
       amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 2));
       amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 1));
       const float qs = __fdiv_rn(fmaxf(amax, 1e-6f), a.upper_max);
-      if (l8 == 0) a.q_scale[static_cast<int64_t>(r.t) * a.Hq + h] = qs;
+      if (l8 == 0) a.q_scale[r.qs + static_cast<int64_t>(h) * (a.qs_prefill ? a.qs_ld : 1)] = qs;
       const float rq = __frcp_rn(qs);
       const float2 b2 = make_float2(qs, qs), r2 = make_float2(rq, rq);
 #pragma unroll
@@ -344,10 +362,13 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
   } else {  // ------------------------------------------------------------ K
     const int kh = h - a.Hq;
     char* page_base = a.k_cache + static_cast<int64_t>(r.page) * a.k_page_bytes;
-    char* dst = page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
+    char* dst = a.out_k != nullptr
+                    ? a.out_k + (static_cast<int64_t>(r.t) * a.Hkv + kh) * kHeadDim * ES
+                    : page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
     if (POLICY != 0) divide_pairs(y, __ldg(a.k_scale));
     store_head<POLICY>(dst, y, l8);
-    if (TAILS && r.is_last) zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
+    if (TAILS && r.is_last && a.out_k == nullptr)
+      zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
   }
 }
 

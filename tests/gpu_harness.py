@@ -104,7 +104,10 @@ def rotation_terms(w, r, head, pos):
     x = bf16_bits_to_f32(w.qkv[r, head * D:(head + 1) * D]).astype(np.float64)
     wts = w.q_norm_w if head < w.Hq else w.k_norm_w
     if wts is not None:
-        y = x / np.sqrt(np.mean(x * x) + w.eps) * bf16_bits_to_f32(wts).astype(np.float64)
+        wf = bf16_bits_to_f32(wts).astype(np.float64)
+        if w.norm_style == 1:         # Gemma-style: 1 + w
+            wf = 1.0 + wf
+        y = x / np.sqrt(np.mean(x * x) + w.eps) * wf
     else:
         y = x
     half = w.rot_dim // 2
@@ -125,9 +128,14 @@ class AppendRun:
     """Device state of one fqr_append_paged call plus what the oracle needs."""
 
     def __init__(self, w, *, fill_seed=11, q_indptr=None, seq_lens=None, page_stride_pad=0,
-                 schedule=0):
+                 schedule=0, null_caches=True):
         self.w = w
         self.schedule = schedule
+        self.owned = bool(w.out_kv)
+        # with caller-owned K/V the caches and the page table are passed as NULL
+        # (unless null_caches is False); the caches still exist here so that
+        # every byte of them can be checked to be untouched
+        self.null_caches = self.owned and null_caches
         self.q_indptr = np.asarray(w.q_indptr if q_indptr is None else q_indptr, np.int32)
         self.seq_lens = np.asarray(w.seq_lens if seq_lens is None else seq_lens, np.int32)
         es = w.kv_esize
@@ -156,7 +164,16 @@ class AppendRun:
         self.out_q = torch.empty((w.T, w.Hq, D), dtype=_dt(w.q_esize), device=DEV)
         fill_random_(self.out_q, fill_seed + 2)
         self.out_q_before = self.out_q.clone()
-        self.q_scale = torch.full((max(w.T, 1), w.Hq), float("nan"), device=DEV)
+        qs_shape = w.q_scale_shape if w.max_seqlen > 0 or w.T > 0 else (1, w.Hq)
+        self.q_scale = torch.full(qs_shape, float("nan"), device=DEV)
+        self.q_scale_before = self.q_scale.clone()
+        if self.owned:
+            self.out_k = torch.empty((w.T, w.Hkv, D), dtype=_dt(es), device=DEV)
+            self.out_v = torch.empty((w.T, w.Hkv, D), dtype=_dt(es), device=DEV)
+            fill_random_(self.out_k, fill_seed + 3)
+            fill_random_(self.out_v, fill_seed + 4)
+            self.out_k_before = self.out_k.clone()
+            self.out_v_before = self.out_v.clone()
         self.flags = torch.full((w.B,), 0x5A5A5A5A, dtype=torch.int32, device=DEV)
         self.scales = {k: torch.tensor([v], dtype=torch.float32, device=DEV)
                        for k, v in (("q_scale_inv", w.q_scale_inv), ("k_scale", w.k_scale),
@@ -170,19 +187,28 @@ class AppendRun:
                     q_scale_inv=self.scales["q_scale_inv"] if w.quant_policy == 2 else None,
                     k_scale=self.scales["k_scale"] if w.quant_policy else None,
                     v_scale=self.scales["v_scale"] if w.quant_policy else None,
-                    upper_max=w.upper_max, schedule=self.schedule)
+                    upper_max=w.upper_max, schedule=self.schedule, max_seqlen=w.max_seqlen,
+                    norm_style=w.norm_style,
+                    out_k=self.out_k if self.owned else None,
+                    out_v=self.out_v if self.owned else None)
 
     def launch(self, stream=None):
-        fqr.append_paged(self.qkv, self.cs, self.indptr_d, self.seq_d, self.pt_d, self.k_cache,
-                         self.v_cache, self.out_q, self.flags, stream=stream, **self.kwargs())
+        nul = self.null_caches
+        fqr.append_paged(self.qkv, self.cs, self.indptr_d, self.seq_d,
+                         None if nul else self.pt_d, None if nul else self.k_cache,
+                         None if nul else self.v_cache, self.out_q, self.flags, stream=stream,
+                         **self.kwargs())
 
     # ------------------------------------------------------------ checking --
     def run_oracle(self):
         w = self.w
         P = w.page_size
         valid = oracle.validate(self.q_indptr, self.seq_lens, w.T, w.max_pages, P,
-                                w.cos_sin_rows, w.positions) == 0
-        pages = touched_pages(w.page_table, self.q_indptr, self.seq_lens, P) if valid else []
+                                w.cos_sin_rows, w.positions,
+                                max_seqlen=w.max_seqlen if w.quant_policy == 1 else 0,
+                                paged=not self.owned) == 0
+        pages = touched_pages(w.page_table, self.q_indptr, self.seq_lens, P) \
+            if valid and not self.owned else []
         remap = {g: i for i, g in enumerate(pages)}
         pt = np.full_like(w.page_table, -1)
         for (b, k), g in np.ndenumerate(w.page_table):
@@ -195,11 +221,22 @@ class AppendRun:
             np.zeros((1, P, w.Hkv, D), _np(self.k_before[:1]).dtype)
         vc = _np(self.v_before[idx, :inner]).reshape(shape).copy() if pages else kc.copy()
         oq = _np(self.out_q_before).copy()
-        qs = np.full((max(w.T, 1), w.Hq), np.nan, np.float32)
+        qs = self.q_scale_before.cpu().numpy().copy()
         fl = np.full(w.B, 0x5A5A5A5A, np.int32)
+        ok = _np(self.out_k_before).copy() if self.owned else None
+        ov = _np(self.out_v_before).copy() if self.owned else None
         rc = oracle.append_paged(w, kc, vc, oq, qs if w.quant_policy == 1 else None, fl,
-                                 page_table=pt, q_indptr=self.q_indptr, seq_lens=self.seq_lens)
-        return dict(rc=rc, pages=pages, idx=idx, k=kc, v=vc, out_q=oq, q_scale=qs, flags=fl)
+                                 page_table=pt, q_indptr=self.q_indptr, seq_lens=self.seq_lens,
+                                 out_k=ok, out_v=ov)
+        return dict(rc=rc, pages=pages, idx=idx, k=kc, v=vc, out_q=oq, q_scale=qs, flags=fl,
+                    out_k=ok, out_v=ov)
+
+    def q_scale_at(self, qs, r, h):
+        """q_scale of packed row r, Q head h, in the call's layout."""
+        if self.w.max_seqlen > 0:
+            b = int(np.searchsorted(self.q_indptr, r, side="right") - 1)
+            return float(qs[b, h, r - int(self.q_indptr[b])])
+        return float(qs[r, h])
 
     def check(self, ref=None, *, exact_frac_min=0.99):
         """Compare the device state with the oracle; returns a small report."""
@@ -217,11 +254,24 @@ class AppendRun:
                                     ("v", self.v_store, self.v_before)):
             extra = changed_pages(after, before) - touched
             assert not extra, f"{name} cache: untouched pages written: {sorted(extra)[:8]}"
+        if self.owned:
+            assert not changed_pages(self.k_store, self.k_before), "k cache written (owned K/V)"
+            assert not changed_pages(self.v_store, self.v_before), "v cache written (owned K/V)"
         if ref["rc"] != 0:   # malformed: nothing but the flags may change
             assert torch.equal(self.out_q, self.out_q_before), "out_q written on a flagged call"
             if w.quant_policy == 1:
                 assert torch.isnan(self.q_scale).all(), "q_scale written on a flagged call"
+            if self.owned:
+                assert torch.equal(self.out_k, self.out_k_before), "out_k written on a flagged call"
+                assert torch.equal(self.out_v, self.out_v_before), "out_v written on a flagged call"
             return {"flagged": True}
+        if self.owned and w.T:
+            og, ovg = _np(self.out_k), _np(self.out_v)
+            assert np.array_equal(ovg, ref["out_v"]), "owned V rows"
+            ulp = ulp_bf16 if w.kv_esize == 2 else ulp_e4m3
+            d = ulp(og, ref["out_k"])
+            rep["k_cond"] = self._conditioned(d, og, ref["out_k"], ref, "k_owned")
+            rep["k_exact_frac"] = float((d == 0).mean())
         # touched pages
         inner = w.page_size * w.Hkv * D
         shape = (len(ref["pages"]),) + tuple(self.k_cache.shape[1:])
@@ -244,8 +294,12 @@ class AppendRun:
             rep["q_exact_frac"] = float((d == 0).mean())
             assert rep["q_exact_frac"] >= exact_frac_min, rep
             if w.quant_policy == 1:
-                qs = self.q_scale[: w.T].cpu().numpy()
-                rel = np.abs(qs - ref["q_scale"][: w.T]) / np.abs(ref["q_scale"][: w.T])
+                qs = self.q_scale.cpu().numpy()
+                want = ref["q_scale"]
+                # entries no token owns (prefill padding) stay untouched
+                assert np.array_equal(np.isnan(qs), np.isnan(want)), "q_scale entries written"
+                m = ~np.isnan(want)
+                rel = np.abs(qs[m] - want[m]) / np.abs(want[m])
                 assert rel.max() <= 1e-5, f"q_scale rel {rel.max()}"
                 rep["q_scale_rel_max"] = float(rel.max())
         return rep
@@ -261,12 +315,15 @@ class AppendRun:
         bf = (w.q_esize if which == "q" else w.kv_esize) == 2
         dec = bf16_bits_to_f32 if bf else e4m3_decode
         spacing = _spacing_bf16 if bf else _spacing_e4m3
-        tokmap = None if which == "q" else self._k_token_map(ref)
+        tokmap = self._k_token_map(ref) if which == "k" else None
         bad = []
         for ix in idx:
             if which == "q":
                 r, h, i = (int(v) for v in ix)
                 head = h
+            elif which == "k_owned":           # out_k [T, Hkv, 128]
+                r, kh, i = (int(v) for v in ix)
+                head = w.Hq + kh
             else:
                 pg, row, kh, i = (int(v) for v in ix)
                 r = tokmap[(pg, row)]
@@ -278,7 +335,7 @@ class AppendRun:
             if which == "q":
                 scale = {0: 1.0, 2: w.q_scale_inv}.get(w.quant_policy)
                 if scale is None:
-                    scale = 1.0 / float(ref["q_scale"][r, h])
+                    scale = 1.0 / self.q_scale_at(ref["q_scale"], r, h)
             else:
                 scale = 1.0 if w.quant_policy == 0 else 1.0 / w.k_scale
             g = float(dec(np.array([got[tuple(ix)]]))[0])

@@ -120,7 +120,18 @@ APPEND_BAD = {
     "fp8_without_kv_scales": dict(quant_policy=2, q_scale_inv=FAKE),
     "fp8_page_stride_unaligned": dict(quant_policy=2, q_scale_inv=FAKE, k_scale=FAKE,
                                       v_scale=FAKE, k_page_stride=16 * 128 + 8),
+    "max_seqlen_negative": dict(max_seqlen=-1),
+    "norm_style_2": dict(norm_style=2),
+    "out_k_without_out_v": dict(out_k=FAKE),
+    "out_v_without_out_k": dict(out_v=FAKE),
+    "misaligned_out_k": dict(out_k=FAKE + 8, out_v=FAKE),
+    "owned_kv_null_cos_sin": dict(out_k=FAKE, out_v=FAKE, cos_sin_cache=None),
 }
+
+# caller-owned K/V rows: the paged caches, the page table and their sizes are
+# not used and may be absent
+OWNED_OK = dict(out_k=FAKE, out_v=FAKE, k_cache=None, v_cache=None, page_table=None,
+                page_size=0, num_pages=0, max_pages=0, k_page_stride=0, v_page_stride=0)
 
 
 @pytest.mark.parametrize("case", sorted(APPEND_BAD))
@@ -130,6 +141,21 @@ def test_append_host_checks_reject(fqr, case):
 
 def test_append_neox_partial_rotary_is_unsupported(fqr):
     assert fqr.append_paged_raw(valid_append(fqr, rot_dim=64)) == fqr.FQR_ENOTSUP
+
+
+def test_append_prefill_q_scale_layout_beyond_32_bit_indexing_is_unsupported(fqr):
+    dyn = dict(quant_policy=1, q_scale=FAKE, k_scale=FAKE, v_scale=FAKE, B=4096, Hq=64,
+               qkv_row_stride=66 * 128, Hkv=1)
+    # 4096 * 64 * 8192 = 2^31 entries
+    assert fqr.append_paged_raw(valid_append(fqr, max_seqlen=8192, **dyn)) == fqr.FQR_ENOTSUP
+
+
+def test_append_owned_kv_needs_no_cache_or_page_table(fqr):
+    """With the checks passed the call would launch, which needs a GPU: every
+    host check must pass and the call must reach the CUDA runtime."""
+    for over in (OWNED_OK, dict(OWNED_OK, norm_style=1),
+                 dict(quant_policy=1, q_scale=FAKE, k_scale=FAKE, v_scale=FAKE, max_seqlen=129)):
+        assert fqr.append_paged_raw(valid_append(fqr, **over)) == fqr.FQR_ECUDA
 
 
 def test_append_null_params(fqr):
