@@ -53,6 +53,8 @@ class _MlaArgs(ctypes.Structure):
         ("block_table", c_vp), ("max_blocks", c_i32),
         ("latent_cache", c_vp), ("num_blocks", c_i32), ("block_size", c_i32),
         ("cache_fp8", c_i32), ("kv_scale", c_f32), ("flags", c_vp),
+        ("q_quant", c_i32), ("q_scale_inv", c_f32), ("upper_max", c_f32),
+        ("q_out", c_vp), ("q_scale", c_vp),
     ]
 
 
@@ -198,12 +200,23 @@ def append_paged(w, k_cache: np.ndarray, v_cache: np.ndarray, out_q: np.ndarray,
     return lib().fqro_append_paged(ctypes.byref(a))
 
 
+def new_mla_q_outputs(w):
+    """q_out [T, Hq, nope + rope] and q_scale ([T] per token, [T, Hq] per
+    head) of the MLA Q quantisation, pre-filled with sentinels."""
+    q_out = np.full((w.T, w.Hq, w.nope_dim + w.rope_dim), 0xFF, np.uint8)
+    shape = {2: (w.T,), 3: (w.T, w.Hq)}.get(w.q_quant, (1,))
+    return q_out, np.full(shape, np.nan, np.float32)
+
+
 def concat_mla_cache(w, q: np.ndarray, latent: np.ndarray, flags: np.ndarray, *,
                      block_table: Optional[np.ndarray] = None,
                      q_indptr: Optional[np.ndarray] = None,
-                     seq_lens: Optional[np.ndarray] = None) -> int:
-    """Run the oracle MLA concat; q [T, Hq, nope+rope] is rotated in place and
-    latent [n_blocks, block_size, rank + rope] receives the rows."""
+                     seq_lens: Optional[np.ndarray] = None,
+                     q_out: Optional[np.ndarray] = None,
+                     q_scale: Optional[np.ndarray] = None) -> int:
+    """Run the oracle MLA concat; q [T, Hq, nope+rope] is rotated in place (or,
+    with w.q_quant, quantised into q_out / q_scale) and latent [n_blocks,
+    block_size, rank + rope] receives the rows."""
     bt = np.ascontiguousarray(w.block_table if block_table is None else block_table,
                               dtype=np.int32)
     ind = np.ascontiguousarray(w.q_indptr if q_indptr is None else q_indptr, dtype=np.int32)
@@ -223,9 +236,11 @@ def concat_mla_cache(w, q: np.ndarray, latent: np.ndarray, flags: np.ndarray, *,
         block_table=_ptr(bt), max_blocks=bt.shape[1],
         latent_cache=_ptr(latent), num_blocks=latent.shape[0],
         block_size=w.block_size, cache_fp8=w.cache_fp8, kv_scale=w.kv_scale,
-        flags=_ptr(flags))
+        flags=_ptr(flags), q_quant=w.q_quant, q_scale_inv=w.q_scale_inv,
+        upper_max=w.upper_max, q_out=_ptr(q_out), q_scale=_ptr(q_scale))
     return lib().fqro_concat_mla_cache(ctypes.byref(a))
 
 
 __all__ = ["lib", "e4m3", "bf16", "bf16_to_f32", "rmsnorm", "rope", "validate",
-           "new_outputs", "new_kv_outputs", "append_paged", "concat_mla_cache"]
+           "new_outputs", "new_kv_outputs", "new_mla_q_outputs", "append_paged",
+           "concat_mla_cache"]

@@ -316,6 +316,43 @@ int fqro_append_paged(const fqro_append_args* a) {
 /* MLA latent concat ([VLLM] concat_and_cache_mla; interleaved RoPE on the    */
 /* rope part of Q and on k_pe; latent row = [kv_c | rope(k_pe)])             */
 /* ------------------------------------------------------------------------ */
+/* The fp32 values v = [nope | rope(rope part)] of head h of row r. */
+static void mla_q_values(const fqro_mla_args* a, int64_t r, int h, const float* cs, float* v) {
+  const uint16_t* qp = a->q + r * a->q_token_stride + h * a->q_head_stride;
+  widen_head(qp, v, a->nope_dim + a->rope_dim);
+  rope(v + a->nope_dim, cs, a->rope_dim, a->rope_style);
+}
+
+/* Q quantisation of row r ([VLLM] "static per-tensor, dynamic per-token, and
+ * dynamic per-group"; the scale and payload forms of the dynamic per-head Q
+ * scale of [FI] "Contract"). */
+static void quantize_q(const fqro_mla_args* a, int64_t r, const float* cs) {
+  const int W = a->nope_dim + a->rope_dim;
+  float v[1024];
+  float s = 0.0f;
+  if (a->q_quant == 2) {  /* one scale for the whole token */
+    float amax = 0.0f;
+    for (int h = 0; h < a->Hq; ++h) {
+      mla_q_values(a, r, h, cs, v);
+      for (int i = 0; i < W; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    }
+    s = fmaxf(amax, 1e-6f) / a->upper_max;
+    a->q_scale[r] = s;
+  }
+  for (int h = 0; h < a->Hq; ++h) {
+    mla_q_values(a, r, h, cs, v);
+    if (a->q_quant == 3) {  /* one scale per head */
+      float amax = 0.0f;
+      for (int i = 0; i < W; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      s = fmaxf(amax, 1e-6f) / a->upper_max;
+      a->q_scale[r * a->Hq + h] = s;
+    }
+    uint8_t* out = a->q_out + (r * a->Hq + h) * W;
+    for (int i = 0; i < W; ++i)
+      out[i] = fqro_f32_to_e4m3_rn_satfinite(a->q_quant == 1 ? v[i] * a->q_scale_inv : v[i] / s);
+  }
+}
+
 int fqro_concat_mla_cache(const fqro_mla_args* a) {
   if (fqro_validate(a->q_indptr, a->seq_lens, a->B, a->T, a->max_blocks,
                     a->block_size, a->cos_sin_rows, a->positions, 0, 1)) {
@@ -324,7 +361,7 @@ int fqro_concat_mla_cache(const fqro_mla_args* a) {
   }
   const int R = a->rope_dim, K = a->kv_lora_rank, W = K + R;
   float y[512];
-  if (R > 512) return 2;
+  if (R > 512 || a->nope_dim + R > 1024) return 2;
   for (int32_t b = 0; b < a->B; ++b) {
     int64_t lo = a->q_indptr[b], hi = a->q_indptr[b + 1], L = a->seq_lens[b];
     for (int64_t r = lo; r < hi; ++r) {
@@ -333,12 +370,16 @@ int fqro_concat_mla_cache(const fqro_mla_args* a) {
       int64_t blk = a->block_table[(int64_t)b * a->max_blocks + p_slot / a->block_size];
       int64_t row = p_slot % a->block_size;
       const float* cs = a->cos_sin + pos * R;
-      /* Q: rotate the rope part in place, the nope part is left as it is */
-      for (int h = 0; h < a->Hq; ++h) {
-        uint16_t* qp = a->q + r * a->q_token_stride + h * a->q_head_stride + a->nope_dim;
-        widen_head(qp, y, R);
-        rope(y, cs, R, a->rope_style);
-        for (int i = 0; i < R; ++i) qp[i] = fqro_f32_to_bf16_rne(y[i]);
+      if (a->q_quant == 0) {
+        /* Q: rotate the rope part in place, the nope part is left as it is */
+        for (int h = 0; h < a->Hq; ++h) {
+          uint16_t* qp = a->q + r * a->q_token_stride + h * a->q_head_stride + a->nope_dim;
+          widen_head(qp, y, R);
+          rope(y, cs, R, a->rope_style);
+          for (int i = 0; i < R; ++i) qp[i] = fqro_f32_to_bf16_rne(y[i]);
+        }
+      } else {
+        quantize_q(a, r, cs);
       }
       /* latent row */
       int64_t base = (blk * a->block_size + row) * W;

@@ -114,6 +114,17 @@ typedef struct {
   int32_t cache_fp8;          /* 1: e4m3 codes (x / kv_scale), 0: bf16 bits   */
   float kv_scale;
   int32_t* flags;             /* [B]                                         */
+  /* Q quantisation: 0 none (rope part rotated in place, BF16); otherwise q is
+   * read-only and q_out [T, Hq, nope + rope] receives e4m3 codes of
+   * v = [nope | rope(rope part)] (fp32):
+   *   1 static per-tensor:     e4m3(v * q_scale_inv)
+   *   2 dynamic per-token:     s = max(max |v| over the token, 1e-6) / upper_max,
+   *                            e4m3(v / s), q_scale [T]
+   *   3 dynamic per-head:      the same with the max over one head, q_scale [T, Hq] */
+  int32_t q_quant;
+  float q_scale_inv, upper_max;
+  uint8_t* q_out;
+  float* q_scale;
 } fqro_mla_args;
 
 int fqro_concat_mla_cache(const fqro_mla_args* a);

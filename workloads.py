@@ -131,6 +131,9 @@ class MlaWorkload:
     block_size: int
     cache_fp8: int
     kv_scale: float
+    q_quant: int = 0           # 0 none, 1 static, 2 dynamic per token, 3 per head
+    q_scale_inv: float = 1.0
+    upper_max: float = 448.0
 
     @property
     def kv_lora_rank(self) -> int:
@@ -254,10 +257,12 @@ def malformed_indptr(w: AppendWorkload, seed=1104) -> np.ndarray:
     return ind
 
 
-def mla_decode(seed=1005) -> MlaWorkload:
+def mla_decode(seed=1005, q_quant=0) -> MlaWorkload:
     """MLA decode latent concat: 32 x 1 token, 128 query heads, q [32,128,192]
     with interleaved RoPE on dims 128..191 (theta 10000), kv_c [32, 512],
-    k_pe [32, 64], FP8 latent cache [16384, 64, 576] with scale 0.02."""
+    k_pe [32, 64], FP8 latent cache [16384, 64, 576] with scale 0.02.
+    q_quant > 0: the same call with Q quantised to FP8 E4M3 (1 static
+    per-tensor with q_scale_inv 1/0.02, 2 dynamic per token, 3 per head)."""
     rng = rng_for(seed)
     B = T = 32
     Hq, nope, rope_dim, rank = 128, 128, 64, 512
@@ -270,18 +275,21 @@ def mla_decode(seed=1005) -> MlaWorkload:
     perm = rng.permutation(num_blocks).astype(np.int32).reshape(B, max_blocks)
     cs = cos_sin_cache(32768, rope_dim, 10000.0)
     q_indptr = np.arange(B + 1, dtype=np.int32)
-    return MlaWorkload(name="mla_decode_B32_h128_latent576_fp8", seed=seed,
+    suffix = {0: "", 1: "_qfp8_static", 2: "_qfp8_token", 3: "_qfp8_head"}[q_quant]
+    return MlaWorkload(name="mla_decode_B32_h128_latent576_fp8" + suffix, seed=seed,
                        T=T, B=B, Hq=Hq, nope_dim=nope, rope_dim=rope_dim, q=q,
                        kv_c=kv_c, k_pe=k_pe, cos_sin=cs, rope_style=1,
                        positions=None, q_indptr=q_indptr, seq_lens=L,
                        block_table=perm.copy(), num_blocks=num_blocks,
-                       block_size=block_size, cache_fp8=1, kv_scale=0.02)
+                       block_size=block_size, cache_fp8=1, kv_scale=0.02,
+                       q_quant=q_quant, q_scale_inv=1 / 0.02)
 
 
 def make_mla(*, seed=0, n_new, seq_lens, Hq, block_size, max_blocks,
              num_blocks=None, nope_dim=128, rope_dim=64, kv_lora_rank=512,
              rope_style=1, theta=10000.0, cos_sin_rows=None, cache_fp8=1,
-             kv_scale=0.02, positions=None) -> MlaWorkload:
+             kv_scale=0.02, positions=None, q_quant=0, q_scale_inv=1.0,
+             upper_max=448.0) -> MlaWorkload:
     rng = rng_for(seed)
     n_new = np.asarray(n_new, dtype=np.int64)
     seq_lens = np.asarray(seq_lens, dtype=np.int32)
@@ -306,7 +314,8 @@ def make_mla(*, seed=0, n_new, seq_lens, Hq, block_size, max_blocks,
                        positions=positions, q_indptr=q_indptr,
                        seq_lens=seq_lens, block_table=table,
                        num_blocks=num_blocks, block_size=block_size,
-                       cache_fp8=cache_fp8, kv_scale=kv_scale)
+                       cache_fp8=cache_fp8, kv_scale=kv_scale, q_quant=q_quant,
+                       q_scale_inv=q_scale_inv, upper_max=upper_max)
 
 
 def prefill_dynq_gemma(seed=1006, q_len=129) -> AppendWorkload:
@@ -355,7 +364,10 @@ APPEND_CONFIGS = {
     "decode_out_kv_bf16": decode_out_kv_bf16,
     "gate_tail_decode_bf16": gate_tail_decode_bf16,
 }
-MLA_CONFIGS = {"mla_decode": mla_decode}
+MLA_CONFIGS = {"mla_decode": mla_decode,
+               "mla_decode_qfp8_static": lambda seed=1005: mla_decode(seed, q_quant=1),
+               "mla_decode_qfp8_token": lambda seed=1005: mla_decode(seed, q_quant=2),
+               "mla_decode_qfp8_head": lambda seed=1005: mla_decode(seed, q_quant=3)}
 
 
 # ---------------------------------------------------------------------------
@@ -405,12 +417,18 @@ def append_bytes(w: AppendWorkload) -> dict:
 
 def mla_bytes(w: MlaWorkload) -> dict:
     T, B = w.T, w.B
-    reads = T * w.Hq * w.rope_dim * 2            # q rope part
+    W = w.nope_dim + w.rope_dim
+    if w.q_quant:   # the whole head read, quantised into q_out (one byte each)
+        reads = T * w.Hq * W * 2
+        writes = T * w.Hq * W + {2: 4 * T, 3: 4 * T * w.Hq}.get(w.q_quant, 0)
+    else:           # the rope part rotated in place
+        reads = T * w.Hq * w.rope_dim * 2
+        writes = T * w.Hq * w.rope_dim * 2
     reads += T * (w.kv_lora_rank + w.rope_dim) * 2
     reads += T * w.rope_dim * 4                  # cos/sin row
     reads += 4 * (B + 1) + 4 * B + 4 * T         # metadata + one table entry per token
     cache_e = 1 if w.cache_fp8 else 2
-    writes = T * w.Hq * w.rope_dim * 2 + T * w.width * cache_e + 4 * B
+    writes += T * w.width * cache_e + 4 * B
     return {"read": int(reads), "write": int(writes), "total": int(reads + writes)}
 
 
