@@ -270,9 +270,10 @@ class AppendBench:
 
 
 class MlaBench:
-    def __init__(self, torch, fqr, device, min_bytes=3 * L2_BYTES, max_replicas=256):
+    def __init__(self, torch, fqr, device, min_bytes=3 * L2_BYTES, max_replicas=256,
+                 name="mla_decode"):
         self.torch, self.fqr, self.dev = torch, fqr, device
-        base = workloads.mla_decode()
+        base = workloads.MLA_CONFIGS[name]()
         self.name = base.name
         per = workloads.mla_bytes(base)["total"]
         self.R = int(min(max_replicas, max(2, math.ceil(min_bytes / per))))
@@ -280,7 +281,10 @@ class MlaBench:
                                                seq_lens=base.seq_lens, Hq=base.Hq,
                                                block_size=base.block_size,
                                                max_blocks=base.max_blocks,
-                                               cos_sin_rows=base.cos_sin_rows)
+                                               cos_sin_rows=base.cos_sin_rows,
+                                               q_quant=base.q_quant,
+                                               q_scale_inv=base.q_scale_inv,
+                                               upper_max=base.upper_max)
                             for r in range(1, self.R)]
         self.bytes = [workloads.mla_bytes(w)["total"] for w in self.ws]
         self.T = base.T
@@ -290,14 +294,24 @@ class MlaBench:
         self.scale = torch.tensor([base.kv_scale], dtype=torch.float32, device=device)
         self.params = []
         self.keep = []
+        self.qsi = torch.tensor([base.q_scale_inv], dtype=torch.float32, device=device)
         for w in self.ws:
             q, kv_c, k_pe = self._d(w.q), self._d(w.kv_c), self._d(w.k_pe)
             ind, sl, bt = self._d(w.q_indptr), self._d(w.seq_lens), self._d(w.block_table)
             flags = torch.empty((w.B,), dtype=torch.int32, device=device)
-            self.keep.append((q, kv_c, k_pe, ind, sl, bt, flags))
+            qq = {}
+            if w.q_quant:   # Q quantised into q_out / q_scale (q read-only)
+                q_out = torch.empty((w.T, w.Hq, w.nope_dim + w.rope_dim), dtype=torch.uint8,
+                                    device=device)
+                q_scale = torch.empty({2: (w.T,), 3: (w.T, w.Hq)}.get(w.q_quant, (1,)),
+                                      dtype=torch.float32, device=device)
+                qq = dict(q_quant=w.q_quant, q_scale_inv=self.qsi, upper_max=w.upper_max,
+                          q_out=q_out, q_scale=q_scale)
+            self.keep.append((q, kv_c, k_pe, ind, sl, bt, flags, qq))
             self.params.append(fqr.mla_params(q, kv_c, k_pe, self.cs, ind, sl, bt, self.latent,
                                               flags, nope_dim=w.nope_dim,
-                                              rope_style=w.rope_style, kv_scale=self.scale))
+                                              rope_style=w.rope_style, kv_scale=self.scale,
+                                              **qq))
 
     _d = AppendBench._d
 
@@ -634,15 +648,18 @@ def measure_per_config(torch, fqr, dev, peak, main_name, steps=20000, warmup=200
             out[name]["us_per_launch_by_schedule"][label] = ms_s * 1e3 / n
         del b
         torch.cuda.empty_cache()
-    m = MlaBench(torch, fqr, dev)
-    n = 20000
-    ms, nbytes = time_launches(torch, m, n, warmup)
-    us = ms * 1e3 / n
-    gbs = nbytes / n / (us * 1e-6) / 1e9
-    out["mla_decode"] = {"workload": m.name, "us_per_launch": us,
-                         "tokens_per_s": m.T / (us * 1e-6), "GB_per_s": gbs,
-                         "frac_of_peak": gbs / peak, "bytes_per_launch": nbytes / n,
-                         "replicas": m.R, "launches": n}
+    for name in workloads.MLA_CONFIGS:
+        m = MlaBench(torch, fqr, dev, name=name)
+        n = 20000
+        ms, nbytes = time_launches(torch, m, n, warmup)
+        us = ms * 1e3 / n
+        gbs = nbytes / n / (us * 1e-6) / 1e9
+        out[name] = {"workload": m.name, "us_per_launch": us,
+                     "tokens_per_s": m.T / (us * 1e-6), "GB_per_s": gbs,
+                     "frac_of_peak": gbs / peak, "bytes_per_launch": nbytes / n,
+                     "replicas": m.R, "launches": n}
+        del m
+        torch.cuda.empty_cache()
     return out
 
 

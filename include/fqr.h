@@ -193,10 +193,25 @@ int fqr_append_paged(const fqr_append_params* p, void* stream);
  * flags as for fqr_append_paged (block_table/max_blocks/block_size play the
  * page table's role); when flagged nothing else is written.
  *
+ * Q quantisation (q_quant != 0; vLLM issue #24678: "static per-tensor,
+ * dynamic per-token, and dynamic per-group" Q scales): q is then read-only,
+ * and with v = [q[r, h, 0:nope] | rope(q[r, h, nope:nope+rope])] in fp32,
+ * q_out[r, h, :] (e4m3 [T, Hq, nope + rope], contiguous) receives
+ *   FQR_MLA_Q_STATIC:   e4m3(v * *q_scale_inv)
+ *   FQR_MLA_Q_TOKEN:    e4m3(v / s), s = max(max |v| over all heads of row r,
+ *                       1e-6) / upper_max, q_scale[r] = s         (fp32 [T])
+ *   FQR_MLA_Q_HEAD:     the same with the max over head h alone,
+ *                       q_scale[r * Hq + h] = s                   (fp32 [T, Hq])
+ *
  * Constraints: rope_dim == 64; nope_dim, q_token_stride, q_head_stride
- * multiples of 4; kv_lora_rank, kv_c_stride multiples of 8; k_pe_stride a
- * multiple of 4; q, kv_c, k_pe, latent_cache 16-byte aligned.
+ * multiples of 4 (of 8 with Q quantisation); kv_lora_rank, kv_c_stride
+ * multiples of 8; k_pe_stride a multiple of 4; q, kv_c, k_pe, latent_cache,
+ * q_out 16-byte aligned.
  */
+#define FQR_MLA_Q_NONE 0
+#define FQR_MLA_Q_STATIC 1
+#define FQR_MLA_Q_TOKEN 2
+#define FQR_MLA_Q_HEAD 3
 typedef struct fqr_mla_params {
   uint16_t* q;                 /* bf16, element (r, h, d) at
                                   r*q_token_stride + h*q_head_stride + d     */
@@ -219,6 +234,11 @@ typedef struct fqr_mla_params {
   int32_t cache_fp8;           /* 1 e4m3, 0 bf16                             */
   const float* kv_scale;       /* device fp32 scalar (cache_fp8 = 1)         */
   int32_t* flags;              /* int32 [B]                                  */
+  int32_t q_quant;             /* FQR_MLA_Q_*                                */
+  const float* q_scale_inv;    /* device fp32 scalar (FQR_MLA_Q_STATIC)      */
+  float upper_max;             /* dynamic modes: finite, in (0, 448]         */
+  void* q_out;                 /* e4m3 [T, Hq, nope + rope] (q_quant != 0)   */
+  float* q_scale;              /* fp32 [T] or [T, Hq] (dynamic modes)        */
 } fqr_mla_params;
 
 int fqr_concat_mla_cache(const fqr_mla_params* p, void* stream);

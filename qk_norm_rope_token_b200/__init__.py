@@ -24,6 +24,7 @@ FQR_OK, FQR_EINVAL, FQR_ENOTSUP, FQR_ECUDA = 0, 1, 2, 3
 SCHEDULE_AUTO, SCHEDULE_LATENCY, SCHEDULE_STREAMING = 0, 1, 2
 FLAG_TIMEOUT = -2
 NORM_RMS, NORM_GEMMA = 0, 1
+MLA_Q_NONE, MLA_Q_STATIC, MLA_Q_TOKEN, MLA_Q_HEAD = 0, 1, 2, 3
 HEAD_DIM = 128
 MAX_BATCH = 16384
 
@@ -60,6 +61,8 @@ class MlaParams(ctypes.Structure):
         ("block_table", c_vp), ("max_blocks", c_i32),
         ("latent_cache", c_vp), ("num_blocks", c_i32), ("block_size", c_i32),
         ("cache_fp8", c_i32), ("kv_scale", c_vp), ("flags", c_vp),
+        ("q_quant", c_i32), ("q_scale_inv", c_vp), ("upper_max", c_f32),
+        ("q_out", c_vp), ("q_scale", c_vp),
     ]
 
 
@@ -191,7 +194,8 @@ def append_paged_from_host(host_in: dict, dev_in: dict, host_out: dict, dev_out:
 
 def mla_params(q, kv_c, k_pe, cos_sin_cache, q_indptr, seq_lens, block_table, latent_cache,
                flags, *, nope_dim: int, rope_style: int = 1, kv_scale=None,
-               positions=None) -> MlaParams:
+               positions=None, q_quant: int = MLA_Q_NONE, q_scale_inv=None,
+               upper_max: float = 448.0, q_out=None, q_scale=None) -> MlaParams:
     T = int(q.shape[0])
     rope_dim = int(k_pe.shape[1]) if k_pe.dim() == 2 else 0
     return MlaParams(
@@ -205,14 +209,17 @@ def mla_params(q, kv_c, k_pe, cos_sin_cache, q_indptr, seq_lens, block_table, la
         max_blocks=int(block_table.shape[1]), latent_cache=_ptr(latent_cache),
         num_blocks=int(latent_cache.shape[0]), block_size=int(latent_cache.shape[1]),
         cache_fp8=1 if latent_cache.element_size() == 1 else 0, kv_scale=_ptr(kv_scale),
-        flags=_ptr(flags))
+        flags=_ptr(flags), q_quant=int(q_quant), q_scale_inv=_ptr(q_scale_inv),
+        upper_max=float(upper_max), q_out=_ptr(q_out), q_scale=_ptr(q_scale))
 
 
 def concat_mla_cache(q, kv_c, k_pe, cos_sin_cache, q_indptr, seq_lens, block_table,
                      latent_cache, flags, *, stream=None, **kw) -> None:
-    """MLA: rotate q[..., nope:nope+64] in place and write [kv_c | rope(k_pe)]
-    rows into latent_cache [num_blocks, block_size, rank + 64] (e4m3 with
-    *kv_scale, or bf16).  Raises FqrError on a host-side argument error."""
+    """MLA: rotate q[..., nope:nope+64] in place (or, with q_quant, quantise
+    [nope | rope(rope part)] into q_out / q_scale) and write [kv_c |
+    rope(k_pe)] rows into latent_cache [num_blocks, block_size, rank + 64]
+    (e4m3 with *kv_scale, or bf16).  Raises FqrError on a host-side argument
+    error."""
     p = mla_params(q, kv_c, k_pe, cos_sin_cache, q_indptr, seq_lens, block_table,
                    latent_cache, flags, **kw)
     rc = concat_mla_cache_raw(p, _stream(stream, latent_cache.device))
@@ -226,4 +233,4 @@ __all__ = ["LIB", "LIB_PATH", "AppendParams", "MlaParams", "FqrError", "strerror
            "concat_mla_cache", "concat_mla_cache_raw", "FQR_OK", "FQR_EINVAL",
            "FQR_ENOTSUP", "FQR_ECUDA", "HEAD_DIM", "MAX_BATCH", "SCHEDULE_AUTO",
            "SCHEDULE_LATENCY", "SCHEDULE_STREAMING", "FLAG_TIMEOUT", "NORM_RMS",
-           "NORM_GEMMA"]
+           "NORM_GEMMA", "MLA_Q_NONE", "MLA_Q_STATIC", "MLA_Q_TOKEN", "MLA_Q_HEAD"]

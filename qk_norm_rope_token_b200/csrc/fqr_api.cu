@@ -101,9 +101,23 @@ int check_mla(const fqr_mla_params* p) {
     if (p->q_token_stride < static_cast<int64_t>(p->Hq) * p->q_head_stride) return FQR_EINVAL;
     if (p->kv_c_stride < p->kv_lora_rank || p->k_pe_stride < p->rope_dim) return FQR_EINVAL;
   }
+  if (p->q_quant < FQR_MLA_Q_NONE || p->q_quant > FQR_MLA_Q_HEAD) return FQR_EINVAL;
+  if (p->q_quant != FQR_MLA_Q_NONE) {
+    if (p->T > 0 && (!p->q_out || !aligned(p->q_out, 16))) return FQR_EINVAL;
+    if (p->q_quant == FQR_MLA_Q_STATIC && !p->q_scale_inv) return FQR_EINVAL;
+    if (p->q_quant != FQR_MLA_Q_STATIC) {
+      if (!p->q_scale || !aligned(p->q_scale, 4)) return FQR_EINVAL;
+      if (!(std::isfinite(p->upper_max) && p->upper_max > 0.0f && p->upper_max <= 448.0f))
+        return FQR_EINVAL;
+    }
+  }
   if (p->rope_dim != 64) return FQR_ENOTSUP;
   if (p->nope_dim % 4 || p->q_token_stride % 4 || p->q_head_stride % 4 || p->kv_lora_rank % 8 ||
       p->kv_c_stride % 8 || p->k_pe_stride % 4)
+    return FQR_ENOTSUP;
+  // quantised Q reads the nope part in 16-byte vectors
+  if (p->q_quant != FQR_MLA_Q_NONE &&
+      (p->nope_dim % 8 || p->q_token_stride % 8 || p->q_head_stride % 8))
     return FQR_ENOTSUP;
   return FQR_OK;
 }

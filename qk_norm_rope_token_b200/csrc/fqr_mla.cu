@@ -13,7 +13,11 @@
 //   * Q tasks (one per row and 4 heads): 8 lanes per head, each holding
 //     elements [4l, 4l+4) and [32+4l, 32+4l+4) of the 64 rope dims, which
 //     covers the NeoX pairs (i, i+32) and the GPT-J pairs (2i, 2i+1) alike.
-#include "fqr_device.cuh"
+// With Q quantisation (mla_quant_kernel) the latent tasks stay warp tasks and
+// a block takes the whole Q of one row at a time (every head, so that the
+// per-token scale can be reduced over the block before any payload store);
+// the 8 lanes of a head also hold its nope part in 16-byte chunks.
+#include "fqr_head.cuh"
 #include "fqr_launch.h"
 
 namespace fqr {
@@ -41,6 +45,11 @@ struct MlaArgs {
   int64_t row_bytes;
   const float* kv_scale;
   int32_t* flags;
+  int q_quant;
+  const float* q_scale_inv;
+  float upper_max;
+  unsigned char* q_out;
+  float* q_scale;
 };
 
 __device__ __forceinline__ uint2 ld_v2(const void* p) {
@@ -76,6 +85,48 @@ __device__ __forceinline__ void mla_rotate(float* y /* A[0..4) B[4..8) */, const
   }
 }
 
+// Latent row of packed row t (request b, slot position p_slot): 32 lanes
+// encode kv_c in 16-byte vectors, 8 lanes rotate k_pe.
+template <int FP8, int STYLE>
+__device__ __forceinline__ void latent_row(const MlaArgs& a, int t, int b, int p_slot,
+                                           const float* row, int lane) {
+  const int64_t blk =
+      __ldg(a.block_table + static_cast<int64_t>(b) * a.max_blocks + p_slot / a.block_size);
+  char* dst = a.latent + (blk * a.block_size + p_slot % a.block_size) * a.row_bytes;
+  const uint16_t* kc = a.kv_c + static_cast<int64_t>(t) * a.kv_c_stride;
+  const float sc = FP8 ? __ldg(a.kv_scale) : 1.0f;
+  for (int c8 = lane; c8 < a.rank / 8; c8 += 32) {
+    const uint4 v = ld_stream_v4(kc + 8 * c8);
+    if (FP8) {
+      float y[8];
+      unpack8(v, y);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) y[k] = __fdiv_rn(y[k], sc);
+      st_v2(dst + 8 * c8, pack8_e4m3(y));
+    } else {
+      st_v4(dst + 16 * c8, v);
+    }
+  }
+  if (lane < kRope / 8) {
+    const uint16_t* kp = a.k_pe + static_cast<int64_t>(t) * a.k_pe_stride;
+    float y[8], c[4], s[4];
+    unpack4(ld_stream_v2(kp + 4 * lane), y);
+    unpack4(ld_stream_v2(kp + kRope / 2 + 4 * lane), y + 4);
+    mla_cos_sin<STYLE>(row, lane, c, s);
+    mla_rotate<STYLE>(y, c, s);
+    const int64_t e0 = a.rank + 4 * lane, e1 = a.rank + kRope / 2 + 4 * lane;
+    if (FP8) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) y[k] = __fdiv_rn(y[k], sc);
+      st_u32(dst + e0, pack4_e4m3(y));
+      st_u32(dst + e1, pack4_e4m3(y + 4));
+    } else {
+      st_v2(dst + 2 * e0, pack4_bf16(y));
+      st_v2(dst + 2 * e1, pack4_bf16(y + 4));
+    }
+  }
+}
+
 template <int FP8, int STYLE>
 __global__ void __launch_bounds__(kThreads) mla_kernel(const MlaArgs a) {
   extern __shared__ int smem[];
@@ -104,41 +155,7 @@ __global__ void __launch_bounds__(kThreads) mla_kernel(const MlaArgs a) {
     const float* row = a.cs + pos * kRope;
 
     if (lat) {
-      const int64_t blk =
-          __ldg(a.block_table + static_cast<int64_t>(b) * a.max_blocks + p_slot / a.block_size);
-      char* dst = a.latent + (blk * a.block_size + p_slot % a.block_size) * a.row_bytes;
-      const uint16_t* kc = a.kv_c + static_cast<int64_t>(t) * a.kv_c_stride;
-      const float sc = FP8 ? __ldg(a.kv_scale) : 1.0f;
-      for (int c8 = lane; c8 < a.rank / 8; c8 += 32) {
-        const uint4 v = ld_stream_v4(kc + 8 * c8);
-        if (FP8) {
-          float y[8];
-          unpack8(v, y);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) y[k] = __fdiv_rn(y[k], sc);
-          st_v2(dst + 8 * c8, pack8_e4m3(y));
-        } else {
-          st_v4(dst + 16 * c8, v);
-        }
-      }
-      if (lane < kRope / 8) {
-        const uint16_t* kp = a.k_pe + static_cast<int64_t>(t) * a.k_pe_stride;
-        float y[8], c[4], s[4];
-        unpack4(ld_stream_v2(kp + 4 * lane), y);
-        unpack4(ld_stream_v2(kp + kRope / 2 + 4 * lane), y + 4);
-        mla_cos_sin<STYLE>(row, lane, c, s);
-        mla_rotate<STYLE>(y, c, s);
-        const int64_t e0 = a.rank + 4 * lane, e1 = a.rank + kRope / 2 + 4 * lane;
-        if (FP8) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) y[k] = __fdiv_rn(y[k], sc);
-          st_u32(dst + e0, pack4_e4m3(y));
-          st_u32(dst + e1, pack4_e4m3(y + 4));
-        } else {
-          st_v2(dst + 2 * e0, pack4_bf16(y));
-          st_v2(dst + 2 * e1, pack4_bf16(y + 4));
-        }
-      }
+      latent_row<FP8, STYLE>(a, t, b, p_slot, row, lane);
     } else {
       const int h = static_cast<int>(qw - static_cast<int64_t>(t) * a.qgroups) * 4 + g;
       if (h < a.Hq) {
@@ -157,6 +174,151 @@ __global__ void __launch_bounds__(kThreads) mla_kernel(const MlaArgs a) {
 
 using MlaKernel = void (*)(const MlaArgs);
 
+// ---------------------------------------------------------------- Q FP8 --
+
+// E4M3 codes of 8 values: x * qsi (static) or x / sc with rc = 1 / sc
+// (dynamic, |x / sc| <= upper_max: div2_bounded, see fqr_head.cuh).
+template <int QMODE>
+__device__ __forceinline__ void quantize8(float* x, float qsi, float sc, float rc) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float2 v = make_float2(x[2 * j], x[2 * j + 1]);
+    v = QMODE == FQR_MLA_Q_STATIC ? mul2(v, make_float2(qsi, qsi))
+                                  : div2_bounded(v, make_float2(sc, sc), make_float2(rc, rc));
+    x[2 * j] = v.x;
+    x[2 * j + 1] = v.y;
+  }
+}
+
+// The rope part of the head at qp, rotated: y[0..4) = elements [4 l8, 4 l8 + 4),
+// y[4..8) = [32 + 4 l8, ...) of the 64 rope dims.
+template <int STYLE>
+__device__ __forceinline__ void rope_part(const uint16_t* qp, int nope, int l8, const float* c,
+                                          const float* s, float* y) {
+  unpack4(ld_stream_v2(qp + nope + 4 * l8), y);
+  unpack4(ld_stream_v2(qp + nope + kRope / 2 + 4 * l8), y + 4);
+  mla_rotate<STYLE>(y, c, s);
+}
+
+// max |v| over this lane's share of the head at qp: nope chunks l8, l8 + 8, ...
+// (8 elements each) and the rotated rope part y.
+__device__ __forceinline__ float lane_amax(const uint16_t* qp, int nchunk, int l8, const float* y) {
+  float m = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(y[k]));
+  for (int k = l8; k < nchunk; k += 8) {
+    float x[8];
+    unpack8(ld_stream_v4(qp + 8 * k), x);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(x[j]));
+  }
+  return m;
+}
+
+// Quantised Q of packed row t, every head, by the whole block: warp w, group
+// g takes heads w*4 + g + 32 i.  Per-token scales are reduced over the block
+// (s_red: one float per warp) before any payload is stored.
+template <int QMODE, int STYLE>
+__device__ void quantize_q_row(const MlaArgs& a, int t, const float* row, float* s_red, int warp,
+                               int lane, int g, int l8, unsigned gmask) {
+  const int W = a.nope + kRope, nchunk = a.nope / 8;
+  float c[4], s[4];
+  mla_cos_sin<STYLE>(row, l8, c, s);
+  const uint16_t* qrow = a.q + static_cast<int64_t>(t) * a.q_tok;
+  unsigned char* orow = a.q_out + static_cast<int64_t>(t) * a.Hq * W;
+  float ts = 0.0f, tr = 0.0f;
+  if (QMODE == FQR_MLA_Q_TOKEN) {
+    float m = 0.0f;
+    for (int h = warp * 4 + g; h - g < a.Hq; h += 4 * kWarps) {
+      if (h < a.Hq) {
+        const uint16_t* qp = qrow + static_cast<int64_t>(h) * a.q_head;
+        float y[8];
+        rope_part<STYLE>(qp, a.nope, l8, c, s, y);
+        m = fmaxf(m, lane_amax(qp, nchunk, l8, y));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) s_red[warp] = m;
+    __syncthreads();
+    m = s_red[0];
+#pragma unroll
+    for (int i = 1; i < kWarps; ++i) m = fmaxf(m, s_red[i]);
+    ts = __fdiv_rn(fmaxf(m, 1e-6f), a.upper_max);
+    tr = __frcp_rn(ts);
+    if (threadIdx.x == 0) a.q_scale[t] = ts;
+    __syncthreads();  // s_red is reused by the block's next row
+  }
+  const float qsi = QMODE == FQR_MLA_Q_STATIC ? __ldg(a.q_scale_inv) : 0.0f;
+  for (int h = warp * 4 + g; h - g < a.Hq; h += 4 * kWarps) {
+    if (h >= a.Hq) continue;  // (the whole group)
+    const uint16_t* qp = qrow + static_cast<int64_t>(h) * a.q_head;
+    unsigned char* op = orow + static_cast<int64_t>(h) * W;
+    float y[8];
+    rope_part<STYLE>(qp, a.nope, l8, c, s, y);
+    float sc = ts, rc = tr;
+    if (QMODE == FQR_MLA_Q_HEAD) {
+      float m = lane_amax(qp, nchunk, l8, y);
+      m = fmaxf(m, __shfl_xor_sync(gmask, m, 4));
+      m = fmaxf(m, __shfl_xor_sync(gmask, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(gmask, m, 1));
+      sc = __fdiv_rn(fmaxf(m, 1e-6f), a.upper_max);
+      rc = __frcp_rn(sc);
+      if (l8 == 0) a.q_scale[static_cast<int64_t>(t) * a.Hq + h] = sc;
+    }
+    for (int k = l8; k < nchunk; k += 8) {
+      float x[8];
+      unpack8(ld_stream_v4(qp + 8 * k), x);
+      quantize8<QMODE>(x, qsi, sc, rc);
+      st_v2(op + 8 * k, pack8_e4m3(x));
+    }
+    quantize8<QMODE>(y, qsi, sc, rc);
+    st_u32(op + a.nope + 4 * l8, pack4_e4m3(y));
+    st_u32(op + a.nope + kRope / 2 + 4 * l8, pack4_e4m3(y + 4));
+  }
+}
+
+template <int QMODE, int FP8, int STYLE>
+__global__ void __launch_bounds__(kThreads) mla_quant_kernel(const MlaArgs a) {
+  extern __shared__ int smem[];
+  int* s_indptr = smem;
+  int* s_seq = s_indptr + a.B + 1;
+  float* s_red = reinterpret_cast<float*>(s_seq + a.B);
+  const int lane = threadIdx.x & 31;
+  const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
+  const int g = lane >> 3, l8 = lane & 7;
+  const unsigned gmask = 0xFFu << (8 * g);
+  const int gwarp = blockIdx.x * kWarps + warp;
+  const int nwarps = gridDim.x * kWarps;
+
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
+               static_cast<int64_t>(a.max_blocks) * a.block_size, a.cs_rows};
+  if (stage_and_validate(m, s_indptr, s_seq)) return;
+
+  for (int t = gwarp; t < a.T; t += nwarps) {  // latent rows: warp tasks
+    const int b = request_of_row(s_indptr, a.B, t);
+    const int p_slot = t + s_seq[b] - s_indptr[b + 1];
+    const int64_t pos = a.positions != nullptr ? a.positions[t] : static_cast<int64_t>(p_slot);
+    latent_row<FP8, STYLE>(a, t, b, p_slot, a.cs + pos * kRope, lane);
+  }
+  for (int t = blockIdx.x; t < a.T; t += gridDim.x) {  // Q rows: block tasks
+    const int b = request_of_row(s_indptr, a.B, t);
+    const int p_slot = t + s_seq[b] - s_indptr[b + 1];
+    const int64_t pos = a.positions != nullptr ? a.positions[t] : static_cast<int64_t>(p_slot);
+    quantize_q_row<QMODE, STYLE>(a, t, a.cs + pos * kRope, s_red, warp, lane, g, l8, gmask);
+  }
+}
+
+template <int QMODE>
+static MlaKernel select_quant(int fp8, int style) {
+  if (fp8) return style == 0 ? mla_quant_kernel<QMODE, 1, 0> : mla_quant_kernel<QMODE, 1, 1>;
+  return style == 0 ? mla_quant_kernel<QMODE, 0, 0> : mla_quant_kernel<QMODE, 0, 1>;
+}
+
+
+
 int launch_mla(const fqr_mla_params& p, cudaStream_t stream) {
   MlaArgs a;
   a.q = p.q; a.q_tok = p.q_token_stride; a.q_head = p.q_head_stride;
@@ -171,7 +333,19 @@ int launch_mla(const fqr_mla_params& p, cudaStream_t stream) {
   a.block_size = p.block_size;
   a.row_bytes = static_cast<int64_t>(p.kv_lora_rank + p.rope_dim) * (p.cache_fp8 ? 1 : 2);
   a.kv_scale = p.kv_scale; a.flags = p.flags;
+  a.q_quant = p.q_quant; a.q_scale_inv = p.q_scale_inv; a.upper_max = p.upper_max;
+  a.q_out = static_cast<unsigned char*>(p.q_out); a.q_scale = p.q_scale;
 
+  if (p.q_quant != FQR_MLA_Q_NONE) {
+    MlaKernel k = p.q_quant == FQR_MLA_Q_STATIC  ? select_quant<FQR_MLA_Q_STATIC>(p.cache_fp8, p.rope_style)
+                  : p.q_quant == FQR_MLA_Q_TOKEN ? select_quant<FQR_MLA_Q_TOKEN>(p.cache_fp8, p.rope_style)
+                                                 : select_quant<FQR_MLA_Q_HEAD>(p.cache_fp8, p.rope_style);
+    // one block per row of Q (the latent rows ride along as warp tasks)
+    const int64_t tasks = static_cast<int64_t>(p.T) * kWarps;
+    const size_t smem = static_cast<size_t>(2 * p.B + 1) * sizeof(int) + kWarps * sizeof(float);
+    return launch_persistent(reinterpret_cast<const void*>(k), tasks, smem, stream,
+                             [&](int grid) { return launch_pdl(k, grid, kThreads, smem, stream, a); });
+  }
   MlaKernel k = p.cache_fp8 ? (p.rope_style == 0 ? mla_kernel<1, 0> : mla_kernel<1, 1>)
                             : (p.rope_style == 0 ? mla_kernel<0, 0> : mla_kernel<0, 1>);
   const int64_t tasks = static_cast<int64_t>(p.T) * (1 + a.qgroups);

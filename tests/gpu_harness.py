@@ -391,12 +391,22 @@ class MlaRun:
         self.latent_before = self.latent.clone()
         self.flags = torch.full((w.B,), 0x5A5A5A5A, dtype=torch.int32, device=DEV)
         self.kv_scale = torch.tensor([w.kv_scale], dtype=torch.float32, device=DEV)
+        self.qq = {}
+        if w.q_quant:   # quantised Q: q_out codes and q_scale, sentinel-filled
+            q_out, q_scale = oracle.new_mla_q_outputs(w)
+            self.q_out = torch.empty(q_out.shape, dtype=torch.uint8, device=DEV)
+            fill_random_(self.q_out, fill_seed + 5)
+            self.q_out_before = self.q_out.clone()
+            self.q_scale = torch.from_numpy(q_scale).to(DEV)
+            self.qsi = torch.tensor([w.q_scale_inv], dtype=torch.float32, device=DEV)
+            self.qq = dict(q_quant=w.q_quant, q_scale_inv=self.qsi, upper_max=w.upper_max,
+                           q_out=self.q_out, q_scale=self.q_scale)
 
     def launch(self, stream=None):
         fqr.concat_mla_cache(self.q, self.kv_c, self.k_pe, self.cs, self.indptr_d, self.seq_d,
                              self.bt_d, self.latent, self.flags, nope_dim=self.w.nope_dim,
                              rope_style=self.w.rope_style, kv_scale=self.kv_scale,
-                             positions=self.pos_d, stream=stream)
+                             positions=self.pos_d, stream=stream, **self.qq)
 
     def check(self):
         w = self.w
@@ -420,22 +430,32 @@ class MlaRun:
             np.zeros((1, bs, w.width), _np(self.latent_before[:1]).dtype)
         q = w.q.copy()
         fl = np.full(w.B, 0x5A5A5A5A, np.int32)
+        qo = _np(self.q_out_before).copy() if w.q_quant else None
+        qs = oracle.new_mla_q_outputs(w)[1] if w.q_quant else None
         rc = oracle.concat_mla_cache(w, q, lat, fl, block_table=bt, q_indptr=self.q_indptr,
-                                     seq_lens=self.seq_lens)
+                                     seq_lens=self.seq_lens, q_out=qo, q_scale=qs)
         torch.cuda.synchronize()
         assert np.array_equal(self.flags.cpu().numpy(), fl), "flags"
         assert np.array_equal(_np(self.kv_c), w.kv_c) and np.array_equal(_np(self.k_pe), w.k_pe)
         extra = changed_pages(self.latent, self.latent_before) - set(blocks)
         assert not extra, f"untouched latent blocks written: {sorted(extra)[:8]}"
         qg = _np(self.q)
+        if w.q_quant:
+            assert np.array_equal(qg, w.q), "q written with Q quantisation"
+            # no norm on this path: identical fp32 expressions -> bitwise codes
+            assert np.array_equal(_np(self.q_out), qo), "q_out codes"
+            assert np.array_equal(self.q_scale.cpu().numpy(), qs, equal_nan=True), "q_scale"
         if rc != 0:
             assert np.array_equal(qg, w.q), "q written on a flagged call"
             return {"flagged": True}
-        # q: nope part bitwise; rope part <= 1 ulp
-        assert np.array_equal(qg[..., : w.nope_dim], w.q[..., : w.nope_dim])
-        d = ulp_bf16(qg[..., w.nope_dim:], q[..., w.nope_dim:])
-        assert d.max() <= 1, f"q rope max ulp {d.max()}"
-        rep = {"q_exact_frac": float((d == 0).mean())}
+        if w.q_quant:
+            rep = {"q_exact_frac": 1.0}
+        else:
+            # q: nope part bitwise; rope part <= 1 ulp
+            assert np.array_equal(qg[..., : w.nope_dim], w.q[..., : w.nope_dim])
+            d = ulp_bf16(qg[..., w.nope_dim:], q[..., w.nope_dim:])
+            assert d.max() <= 1, f"q rope max ulp {d.max()}"
+            rep = {"q_exact_frac": float((d == 0).mean())}
         if blocks:
             lg = _np(self.latent[idx])
             written = np.zeros(lg.shape[:2], bool)

@@ -1,6 +1,7 @@
 """GPU parity of fqr_concat_mla_cache against the oracle, through the C ABI:
 the full-size MLA decode workload, BF16 and NeoX variants, ragged prefill
-with empty requests, and malformed metadata."""
+with empty requests, malformed metadata, and Q quantised to FP8 (static,
+per token, per head; bitwise codes and scales)."""
 import numpy as np
 import pytest
 import torch
@@ -71,3 +72,34 @@ def test_mla_graph_replay_matches_eager():
         torch.cuda.synchronize()
         assert torch.equal(r.q, eager_q) and torch.equal(r.latent, eager_lat)
     del g
+
+
+@pytest.mark.parametrize("q_quant", [1, 2, 3])
+def test_mla_decode_q_fp8_parity(q_quant):
+    run(workloads.mla_decode(q_quant=q_quant))
+
+
+@pytest.mark.parametrize("q_quant", [1, 2, 3])
+@pytest.mark.parametrize("style", [1, 0])
+@pytest.mark.parametrize("upper", [448.0, 240.0])
+def test_mla_q_fp8_ragged(q_quant, style, upper):
+    rng = np.random.default_rng(q_quant * 4 + style)
+    B = 7
+    n = rng.integers(0, 30, B)
+    n[2] = 0
+    L = rng.integers(0, 100, B) + n
+    w = workloads.make_mla(seed=9 + q_quant, n_new=n, seq_lens=L, Hq=37, block_size=16,
+                           max_blocks=int(np.ceil(L.max() / 16)) + 1, rope_style=style,
+                           nope_dim=64, kv_lora_rank=256, cos_sin_rows=int(L.max()) + 1,
+                           q_quant=q_quant, q_scale_inv=25.0, upper_max=upper)
+    w.q[0] = 0                                  # an all-zero token (floor scale)
+    run(w)
+
+
+@pytest.mark.parametrize("q_quant", [1, 2, 3])
+def test_mla_q_fp8_malformed_writes_nothing(q_quant):
+    w = workloads.make_mla(seed=4, n_new=[2, 1, 1], seq_lens=[4, 3, 2], Hq=8, block_size=4,
+                           max_blocks=2, kv_lora_rank=64, cos_sin_rows=8, q_quant=q_quant)
+    r, rep = run(w, q_indptr=np.array([0, 3, 2, 4], np.int32))
+    assert rep == {"flagged": True}
+    assert torch.equal(r.q_out, r.q_out_before)
