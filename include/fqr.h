@@ -204,7 +204,8 @@ int fqr_append_paged(const fqr_append_params* p, void* stream);
  *                       q_scale[r * Hq + h] = s                   (fp32 [T, Hq])
  *
  * Constraints: rope_dim == 64; nope_dim, q_token_stride, q_head_stride
- * multiples of 4 (of 8 with Q quantisation); kv_lora_rank, kv_c_stride
+ * multiples of 4 (of 8, and nope_dim <= 256, with Q quantisation);
+ * kv_lora_rank, kv_c_stride
  * multiples of 8; k_pe_stride a multiple of 4; q, kv_c, k_pe, latent_cache,
  * q_out 16-byte aligned.
  */

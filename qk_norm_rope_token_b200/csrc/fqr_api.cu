@@ -115,9 +115,10 @@ int check_mla(const fqr_mla_params* p) {
   if (p->nope_dim % 4 || p->q_token_stride % 4 || p->q_head_stride % 4 || p->kv_lora_rank % 8 ||
       p->kv_c_stride % 8 || p->k_pe_stride % 4)
     return FQR_ENOTSUP;
-  // quantised Q reads the nope part in 16-byte vectors
+  // quantised Q keeps a head's nope part (at most 256 dims) in registers,
+  // loaded in 16-byte vectors
   if (p->q_quant != FQR_MLA_Q_NONE &&
-      (p->nope_dim % 8 || p->q_token_stride % 8 || p->q_head_stride % 8))
+      (p->nope_dim % 8 || p->nope_dim > 256 || p->q_token_stride % 8 || p->q_head_stride % 8))
     return FQR_ENOTSUP;
   return FQR_OK;
 }

@@ -33,6 +33,10 @@ constexpr int kPipeThreads = (kConsumers + 1) * 32;
 constexpr int kMaxStages = 8;
 constexpr int kFixedSmem = 1280;  // barriers (128) + fp32 weights (1024) + spare
 constexpr int kHeader = 32;       // stage header bytes (keeps the copies 16-byte aligned)
+// A NeoX cos/sin row (512 bytes) is staged as four 128-byte quarters with 16
+// bytes between them (kCsPadded in fqr_head.cuh), which makes the lanes'
+// 32-byte slices of it fall on distinct bank groups.
+constexpr uint32_t kCsQuarter = 128;
 
 // Stage header, written by the producer before it arrives on "full".
 struct StageInfo {
@@ -99,6 +103,7 @@ __device__ __forceinline__ void issue_heads(const PipeArgs& a, unsigned char* st
 }
 
 // ------------------------------------------------------------- producer --
+template <int STYLE>
 __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full,
                         uint64_t* empty, const int* s_indptr, const int* s_seq, int64_t u0,
                         int nunits, int pre) {
@@ -145,9 +150,17 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
             ++issued;
           }
           if (csj) {
-            const uint32_t cb = static_cast<uint32_t>(a.hp.rot) * 4;
-            mbar_expect_tx(fb, cb);
-            bulk_g2s(st + kHeader, a.cs + static_cast<int64_t>(posj) * a.hp.rot, cb, fb);
+            const float* src = a.cs + static_cast<int64_t>(posj) * a.hp.rot;
+            if (STYLE == 0) {  // NeoX rows: four 128-byte quarters, 16 bytes apart (kCsPadded)
+              mbar_expect_tx(fb, 4 * kCsQuarter);
+              for (int k = 0; k < 4; ++k)
+                bulk_g2s(st + kHeader + k * (kCsQuarter + 16), src + k * (kCsQuarter / 4),
+                         kCsQuarter, fb);
+            } else {
+              const uint32_t cb = static_cast<uint32_t>(a.hp.rot) * 4;
+              mbar_expect_tx(fb, cb);
+              bulk_g2s(st + kHeader, src, cb, fb);
+            }
           }
         }
       }
@@ -302,7 +315,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) pipe_append_kernel(const Pipe
   }
 
   if (producer) {
-    produce(a, stages, full, empty, s_indptr, s_seq, u0, nunits, pre);
+    produce<STYLE>(a, stages, full, empty, s_indptr, s_seq, u0, nunits, pre);
   } else {
     zero_empty_request_tails<POLICY>(a, s_indptr, s_seq);
     if constexpr (STYLE == 0) {  // NeoX rows are 128 wide: always staged
@@ -342,7 +355,7 @@ int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStr
   a.cs = p.cos_sin_cache;
   a.cs_rows = p.cos_sin_rows;
   a.cs_bulk = (p.rot_dim * 4) % 16 == 0 ? 1 : 0;
-  a.cs_bytes = a.cs_bulk ? p.rot_dim * 4 : 0;
+  a.cs_bytes = !a.cs_bulk ? 0 : p.rope_style == 0 ? kCsPaddedBytes : p.rot_dim * 4;
   a.positions = p.positions;
   a.q_indptr = p.q_indptr;
   a.seq_lens = p.seq_lens;

@@ -194,17 +194,28 @@ __device__ __forceinline__ void zero_tail_column(char* page_base, int row0, int 
   }
 }
 
+// A NeoX cos/sin row staged in shared memory is four 128-byte quarters
+// (cos 0-31, cos 32-63, sin 0-31, sin 32-63), each followed by 16 bytes of
+// padding: lane l8's 32-byte slice starts at quarter l8/4, byte 32*(l8%4),
+// and the 8 lanes of a quarter-warp phase hit 8 distinct 16-byte bank groups.
+constexpr int kCsPaddedBytes = 4 * (128 + 16);
+__device__ __forceinline__ int cs_padded_slice(int l8) { return (l8 >> 2) * 36 + (l8 & 3) * 8; }
+
 // The cos/sin values lane l8 needs for its 8 pairs: NeoX (rot 128) pairs
 // (8l+k, 64+8l+k); GPT-J pairs 4l+j (chunk A) and 32+4l+j (chunk B), with
-// c = s = 0 outside the rotated dims (those pairs are not rotated).
+// c = s = 0 outside the rotated dims (those pairs are not rotated).  A NeoX
+// row in shared memory (CS_SMEM) has the padded layout above; a GPT-J one is
+// contiguous.
 template <int STYLE, bool CS_SMEM>
 __device__ __forceinline__ void load_cs(const float* cs_row, int rot, int l8, float2* c,
                                         float2* s) {
   if (STYLE == 0) {
-    const float4 c0 = ld_cs4<CS_SMEM>(cs_row + 8 * l8);
-    const float4 c1 = ld_cs4<CS_SMEM>(cs_row + 8 * l8 + 4);
-    const float4 s0 = ld_cs4<CS_SMEM>(cs_row + 64 + 8 * l8);
-    const float4 s1 = ld_cs4<CS_SMEM>(cs_row + 68 + 8 * l8);
+    const int i0 = CS_SMEM ? cs_padded_slice(l8) : 8 * l8;  // cos slice
+    const int is = CS_SMEM ? 72 : 64;                        // sin: two quarters on
+    const float4 c0 = ld_cs4<CS_SMEM>(cs_row + i0);
+    const float4 c1 = ld_cs4<CS_SMEM>(cs_row + i0 + 4);
+    const float4 s0 = ld_cs4<CS_SMEM>(cs_row + is + i0);
+    const float4 s1 = ld_cs4<CS_SMEM>(cs_row + is + i0 + 4);
     c[0] = make_float2(c0.x, c0.y); c[1] = make_float2(c0.z, c0.w);
     c[2] = make_float2(c1.x, c1.y); c[3] = make_float2(c1.z, c1.w);
     s[0] = make_float2(s0.x, s0.y); s[1] = make_float2(s0.z, s0.w);

@@ -13,10 +13,11 @@
 //   * Q tasks (one per row and 4 heads): 8 lanes per head, each holding
 //     elements [4l, 4l+4) and [32+4l, 32+4l+4) of the 64 rope dims, which
 //     covers the NeoX pairs (i, i+32) and the GPT-J pairs (2i, 2i+1) alike.
-// With Q quantisation (mla_quant_kernel) the latent tasks stay warp tasks and
-// a block takes the whole Q of one row at a time (every head, so that the
-// per-token scale can be reduced over the block before any payload store);
-// the 8 lanes of a head also hold its nope part in 16-byte chunks.
+// With Q quantisation the 8 lanes of a head also hold its nope part in
+// 16-byte chunks: static and per-head scales keep the warp tasks
+// (mla_quant_kernel); per-token scales give a block of up to 32 warps a whole
+// row of Q at a time (mla_token_kernel), its maximum reduced over the block
+// before any payload store.
 #include "fqr_head.cuh"
 #include "fqr_launch.h"
 
@@ -200,96 +201,71 @@ __device__ __forceinline__ void rope_part(const uint16_t* qp, int nope, int l8, 
   mla_rotate<STYLE>(y, c, s);
 }
 
-// max |v| over this lane's share of the head at qp: nope chunks l8, l8 + 8, ...
-// (8 elements each) and the rotated rope part y.
-__device__ __forceinline__ float lane_amax(const uint16_t* qp, int nchunk, int l8, const float* y) {
+// Quantisation of head h = quad*4 + g of packed row t (Q FP8).  The lane
+// holds the head's nope chunks l8, l8 + 8, ... (8 elements each, kept as
+// packed bf16: at most kMaxChunks) and its rotated rope part y.
+constexpr int kMaxChunks = 4;  // nope_dim <= 256
+
+struct QHead {
+  uint4 nope[kMaxChunks];
+  float y[8];
+};
+
+template <int STYLE>
+__device__ __forceinline__ void load_q_head(const uint16_t* qp, int nope, int l8, const float* c,
+                                            const float* s, QHead& v) {
+#pragma unroll
+  for (int k = 0; k < kMaxChunks; ++k)
+    if (l8 + 8 * k < nope / 8) v.nope[k] = ld_stream_v4(qp + 8 * (l8 + 8 * k));
+  rope_part<STYLE>(qp, nope, l8, c, s, v.y);
+}
+
+__device__ __forceinline__ float q_head_amax(const QHead& v, int nope, int l8) {
   float m = 0.0f;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(y[k]));
-  for (int k = l8; k < nchunk; k += 8) {
-    float x[8];
-    unpack8(ld_stream_v4(qp + 8 * k), x);
+  for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(v.y[k]));
 #pragma unroll
-    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(x[j]));
+  for (int k = 0; k < kMaxChunks; ++k) {
+    if (l8 + 8 * k < nope / 8) {
+      float x[8];
+      unpack8(v.nope[k], x);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(x[j]));
+    }
   }
   return m;
 }
 
-// Quantised Q of packed row t, every head, by the whole block: warp w, group
-// g takes heads w*4 + g + 32 i.  Per-token scales are reduced over the block
-// (s_red: one float per warp) before any payload is stored.
-template <int QMODE, int STYLE>
-__device__ void quantize_q_row(const MlaArgs& a, int t, const float* row, float* s_red, int warp,
-                               int lane, int g, int l8, unsigned gmask) {
-  const int W = a.nope + kRope, nchunk = a.nope / 8;
-  float c[4], s[4];
-  mla_cos_sin<STYLE>(row, l8, c, s);
-  const uint16_t* qrow = a.q + static_cast<int64_t>(t) * a.q_tok;
-  unsigned char* orow = a.q_out + static_cast<int64_t>(t) * a.Hq * W;
-  float ts = 0.0f, tr = 0.0f;
-  if (QMODE == FQR_MLA_Q_TOKEN) {
-    float m = 0.0f;
-    for (int h = warp * 4 + g; h - g < a.Hq; h += 4 * kWarps) {
-      if (h < a.Hq) {
-        const uint16_t* qp = qrow + static_cast<int64_t>(h) * a.q_head;
-        float y[8];
-        rope_part<STYLE>(qp, a.nope, l8, c, s, y);
-        m = fmaxf(m, lane_amax(qp, nchunk, l8, y));
-      }
-    }
+template <int QMODE>
+__device__ __forceinline__ void store_q_head(QHead& v, unsigned char* op, int nope, int l8,
+                                             float qsi, float sc, float rc) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) s_red[warp] = m;
-    __syncthreads();
-    m = s_red[0];
-#pragma unroll
-    for (int i = 1; i < kWarps; ++i) m = fmaxf(m, s_red[i]);
-    ts = __fdiv_rn(fmaxf(m, 1e-6f), a.upper_max);
-    tr = __frcp_rn(ts);
-    if (threadIdx.x == 0) a.q_scale[t] = ts;
-    __syncthreads();  // s_red is reused by the block's next row
-  }
-  const float qsi = QMODE == FQR_MLA_Q_STATIC ? __ldg(a.q_scale_inv) : 0.0f;
-  for (int h = warp * 4 + g; h - g < a.Hq; h += 4 * kWarps) {
-    if (h >= a.Hq) continue;  // (the whole group)
-    const uint16_t* qp = qrow + static_cast<int64_t>(h) * a.q_head;
-    unsigned char* op = orow + static_cast<int64_t>(h) * W;
-    float y[8];
-    rope_part<STYLE>(qp, a.nope, l8, c, s, y);
-    float sc = ts, rc = tr;
-    if (QMODE == FQR_MLA_Q_HEAD) {
-      float m = lane_amax(qp, nchunk, l8, y);
-      m = fmaxf(m, __shfl_xor_sync(gmask, m, 4));
-      m = fmaxf(m, __shfl_xor_sync(gmask, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(gmask, m, 1));
-      sc = __fdiv_rn(fmaxf(m, 1e-6f), a.upper_max);
-      rc = __frcp_rn(sc);
-      if (l8 == 0) a.q_scale[static_cast<int64_t>(t) * a.Hq + h] = sc;
-    }
-    for (int k = l8; k < nchunk; k += 8) {
+  for (int k = 0; k < kMaxChunks; ++k) {
+    const int c = l8 + 8 * k;
+    if (c < nope / 8) {
       float x[8];
-      unpack8(ld_stream_v4(qp + 8 * k), x);
+      unpack8(v.nope[k], x);
       quantize8<QMODE>(x, qsi, sc, rc);
-      st_v2(op + 8 * k, pack8_e4m3(x));
+      st_v2(op + 8 * c, pack8_e4m3(x));
     }
-    quantize8<QMODE>(y, qsi, sc, rc);
-    st_u32(op + a.nope + 4 * l8, pack4_e4m3(y));
-    st_u32(op + a.nope + kRope / 2 + 4 * l8, pack4_e4m3(y + 4));
   }
+  quantize8<QMODE>(v.y, qsi, sc, rc);
+  st_u32(op + nope + 4 * l8, pack4_e4m3(v.y));
+  st_u32(op + nope + kRope / 2 + 4 * l8, pack4_e4m3(v.y + 4));
 }
 
+// Static and per-head scales: persistent warp tasks [latent rows | row x quad].
 template <int QMODE, int FP8, int STYLE>
 __global__ void __launch_bounds__(kThreads) mla_quant_kernel(const MlaArgs a) {
   extern __shared__ int smem[];
   int* s_indptr = smem;
   int* s_seq = s_indptr + a.B + 1;
-  float* s_red = reinterpret_cast<float*>(s_seq + a.B);
   const int lane = threadIdx.x & 31;
   const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
   const int g = lane >> 3, l8 = lane & 7;
   const unsigned gmask = 0xFFu << (8 * g);
-  const int gwarp = blockIdx.x * kWarps + warp;
-  const int nwarps = gridDim.x * kWarps;
+  const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
 
   grid_dependency_wait();
   grid_launch_dependents();
@@ -297,17 +273,120 @@ __global__ void __launch_bounds__(kThreads) mla_quant_kernel(const MlaArgs a) {
                static_cast<int64_t>(a.max_blocks) * a.block_size, a.cs_rows};
   if (stage_and_validate(m, s_indptr, s_seq)) return;
 
-  for (int t = gwarp; t < a.T; t += nwarps) {  // latent rows: warp tasks
+  const int W = a.nope + kRope;
+  const float qsi = QMODE == FQR_MLA_Q_STATIC ? __ldg(a.q_scale_inv) : 0.0f;
+  const int64_t n_tasks = a.T + static_cast<int64_t>(a.T) * a.qgroups;
+  for (int64_t w = gwarp; w < n_tasks; w += nwarps) {
+    const bool lat = w < a.T;
+    const int64_t qw = w - a.T;
+    const int t = lat ? static_cast<int>(w) : static_cast<int>(qw / a.qgroups);
+    const int b = request_of_row(s_indptr, a.B, t);
+    const int p_slot = t + s_seq[b] - s_indptr[b + 1];
+    const int64_t pos = a.positions != nullptr ? a.positions[t] : static_cast<int64_t>(p_slot);
+    const float* row = a.cs + pos * kRope;
+    if (lat) {
+      latent_row<FP8, STYLE>(a, t, b, p_slot, row, lane);
+      continue;
+    }
+    const int h = static_cast<int>(qw - static_cast<int64_t>(t) * a.qgroups) * 4 + g;
+    if (h >= a.Hq) continue;  // (the whole group)
+    float c[4], s[4];
+    mla_cos_sin<STYLE>(row, l8, c, s);
+    QHead v;
+    load_q_head<STYLE>(a.q + static_cast<int64_t>(t) * a.q_tok + static_cast<int64_t>(h) * a.q_head,
+                       a.nope, l8, c, s, v);
+    float sc = 0.0f, rc = 0.0f;
+    if (QMODE == FQR_MLA_Q_HEAD) {
+      float mx = q_head_amax(v, a.nope, l8);
+      mx = fmaxf(mx, __shfl_xor_sync(gmask, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(gmask, mx, 2));
+      mx = fmaxf(mx, __shfl_xor_sync(gmask, mx, 1));
+      sc = __fdiv_rn(fmaxf(mx, 1e-6f), a.upper_max);
+      rc = __frcp_rn(sc);
+      if (l8 == 0) a.q_scale[static_cast<int64_t>(t) * a.Hq + h] = sc;
+    }
+    store_q_head<QMODE>(v, a.q_out + (static_cast<int64_t>(t) * a.Hq + h) * W, a.nope, l8, qsi,
+                        sc, rc);
+  }
+}
+
+// Per-token scales: one block of up to 16 warps per row of Q at a time (each
+// warp's first two quads of heads held in registers), the row's maximum
+// reduced over the block before any payload store; the latent rows are warp
+// tasks first.
+constexpr int kTokenWarps = 16;
+
+template <int FP8, int STYLE>
+__global__ void __launch_bounds__(kTokenWarps * 32) mla_token_kernel(const MlaArgs a) {
+  extern __shared__ int smem[];
+  int* s_indptr = smem;
+  int* s_seq = s_indptr + a.B + 1;
+  float* s_red = reinterpret_cast<float*>(s_seq + a.B);  // one float per warp
+  const int lane = threadIdx.x & 31;
+  const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
+  const int nw = blockDim.x >> 5;
+  const int g = lane >> 3, l8 = lane & 7;
+  const int gwarp = blockIdx.x * nw + warp;
+  const int nwarps = gridDim.x * nw;
+
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
+               static_cast<int64_t>(a.max_blocks) * a.block_size, a.cs_rows};
+  if (stage_and_validate(m, s_indptr, s_seq)) return;
+
+  for (int t = gwarp; t < a.T; t += nwarps) {  // latent rows
     const int b = request_of_row(s_indptr, a.B, t);
     const int p_slot = t + s_seq[b] - s_indptr[b + 1];
     const int64_t pos = a.positions != nullptr ? a.positions[t] : static_cast<int64_t>(p_slot);
     latent_row<FP8, STYLE>(a, t, b, p_slot, a.cs + pos * kRope, lane);
   }
-  for (int t = blockIdx.x; t < a.T; t += gridDim.x) {  // Q rows: block tasks
+  const int W = a.nope + kRope;
+  for (int t = blockIdx.x; t < a.T; t += gridDim.x) {  // Q rows (block-uniform loop)
     const int b = request_of_row(s_indptr, a.B, t);
     const int p_slot = t + s_seq[b] - s_indptr[b + 1];
     const int64_t pos = a.positions != nullptr ? a.positions[t] : static_cast<int64_t>(p_slot);
-    quantize_q_row<QMODE, STYLE>(a, t, a.cs + pos * kRope, s_red, warp, lane, g, l8, gmask);
+    float c[4], s[4];
+    mla_cos_sin<STYLE>(a.cs + pos * kRope, l8, c, s);
+    const uint16_t* qrow = a.q + static_cast<int64_t>(t) * a.q_tok;
+    // pass 1: the row's maximum.  The warp's first two quads are loaded
+    // together and stay in registers; any further quads are read again.
+    const int hA = warp * 4 + g, hB = hA + 4 * nw;
+    const bool okA = hA < a.Hq, okB = hB < a.Hq;  // (group-uniform)
+    QHead va, vb;
+    if (okA) load_q_head<STYLE>(qrow + static_cast<int64_t>(hA) * a.q_head, a.nope, l8, c, s, va);
+    if (okB) load_q_head<STYLE>(qrow + static_cast<int64_t>(hB) * a.q_head, a.nope, l8, c, s, vb);
+    float mx = 0.0f;
+    if (okA) mx = q_head_amax(va, a.nope, l8);
+    if (okB) mx = fmaxf(mx, q_head_amax(vb, a.nope, l8));
+    for (int h = hA + 8 * nw; h - g < a.Hq; h += 4 * nw) {
+      if (h < a.Hq) {
+        QHead v;
+        load_q_head<STYLE>(qrow + static_cast<int64_t>(h) * a.q_head, a.nope, l8, c, s, v);
+        mx = fmaxf(mx, q_head_amax(v, a.nope, l8));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) s_red[warp] = mx;
+    __syncthreads();
+    mx = s_red[0];
+    for (int i = 1; i < nw; ++i) mx = fmaxf(mx, s_red[i]);
+    const float sc = __fdiv_rn(fmaxf(mx, 1e-6f), a.upper_max);
+    const float rc = __frcp_rn(sc);
+    if (threadIdx.x == 0) a.q_scale[t] = sc;
+    // pass 2: payloads
+    unsigned char* orow = a.q_out + static_cast<int64_t>(t) * a.Hq * W;
+    if (okA) store_q_head<FQR_MLA_Q_TOKEN>(va, orow + static_cast<int64_t>(hA) * W, a.nope, l8, 0.0f, sc, rc);
+    if (okB) store_q_head<FQR_MLA_Q_TOKEN>(vb, orow + static_cast<int64_t>(hB) * W, a.nope, l8, 0.0f, sc, rc);
+    for (int h = hA + 8 * nw; h - g < a.Hq; h += 4 * nw) {
+      if (h < a.Hq) {
+        QHead v;
+        load_q_head<STYLE>(qrow + static_cast<int64_t>(h) * a.q_head, a.nope, l8, c, s, v);
+        store_q_head<FQR_MLA_Q_TOKEN>(v, orow + static_cast<int64_t>(h) * W, a.nope, l8, 0.0f, sc, rc);
+      }
+    }
+    __syncthreads();  // s_red is reused by the block's next row
   }
 }
 
@@ -336,13 +415,32 @@ int launch_mla(const fqr_mla_params& p, cudaStream_t stream) {
   a.q_quant = p.q_quant; a.q_scale_inv = p.q_scale_inv; a.upper_max = p.upper_max;
   a.q_out = static_cast<unsigned char*>(p.q_out); a.q_scale = p.q_scale;
 
+  if (p.q_quant == FQR_MLA_Q_TOKEN) {
+    MlaKernel k = p.cache_fp8 ? (p.rope_style == 0 ? mla_token_kernel<1, 0> : mla_token_kernel<1, 1>)
+                              : (p.rope_style == 0 ? mla_token_kernel<0, 0> : mla_token_kernel<0, 1>);
+    const int nw = a.qgroups < kTokenWarps ? a.qgroups : kTokenWarps;  // warps per block
+    const size_t smem = static_cast<size_t>(2 * p.B + 1) * sizeof(int) + nw * sizeof(float);
+    int dev = 0, sms = 0, per_sm = 0;
+    const void* fn = reinterpret_cast<const void*>(k);
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FQR_ECUDA;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return FQR_ECUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 32 * nw, smem) != cudaSuccess ||
+        per_sm < 1)
+      return FQR_ECUDA;
+    const int64_t cap = static_cast<int64_t>(per_sm) * sms;
+    const int64_t want = p.T > 0 ? p.T : 1;
+    return launch_pdl(k, static_cast<int>(want < cap ? want : cap), 32 * nw, smem, stream, a);
+  }
   if (p.q_quant != FQR_MLA_Q_NONE) {
-    MlaKernel k = p.q_quant == FQR_MLA_Q_STATIC  ? select_quant<FQR_MLA_Q_STATIC>(p.cache_fp8, p.rope_style)
-                  : p.q_quant == FQR_MLA_Q_TOKEN ? select_quant<FQR_MLA_Q_TOKEN>(p.cache_fp8, p.rope_style)
-                                                 : select_quant<FQR_MLA_Q_HEAD>(p.cache_fp8, p.rope_style);
-    // one block per row of Q (the latent rows ride along as warp tasks)
-    const int64_t tasks = static_cast<int64_t>(p.T) * kWarps;
-    const size_t smem = static_cast<size_t>(2 * p.B + 1) * sizeof(int) + kWarps * sizeof(float);
+    MlaKernel k = p.q_quant == FQR_MLA_Q_STATIC ? select_quant<FQR_MLA_Q_STATIC>(p.cache_fp8, p.rope_style)
+                                                : select_quant<FQR_MLA_Q_HEAD>(p.cache_fp8, p.rope_style);
+    const int64_t tasks = static_cast<int64_t>(p.T) * (1 + a.qgroups);
+    const size_t smem = static_cast<size_t>(2 * p.B + 1) * sizeof(int);
     return launch_persistent(reinterpret_cast<const void*>(k), tasks, smem, stream,
                              [&](int grid) { return launch_pdl(k, grid, kThreads, smem, stream, a); });
   }
