@@ -18,9 +18,9 @@
 //   * consumer warps take 4 heads at a time from the stage (fqr_head.cuh),
 //     store straight to out_q / the cache slot and release the stage on its
 //     "empty" mbarrier; the quad -> warp assignment rotates every unit.
-//   * the K/V heads of a request's last row zero their column of the tail
-//     rows; consumer warps of the grid zero the tails of requests that append
-//     nothing.
+//   * the 8 consumer warps split the last-page tail of a request's last row
+//     evenly between them (after releasing the stage); consumer warps of the
+//     grid zero the tails of requests that append nothing.
 //   * every block validates the whole batch first; every wait is bounded
 //     (kWaitLimitNs) and a wait that gives up sets every flag to kFlagTimeout.
 #include "fqr_head.cuh"
@@ -47,6 +47,7 @@ static_assert(sizeof(StageInfo) <= kHeader, "stage header");
 struct PipeArgs {
   HeadParams hp;
   FastDiv cdiv;  // division by nchunks
+  FastDiv wdiv;  // division by kConsumers (tail shares)
   const uint16_t* qkv;
   int64_t row_stride;
   int T, B, H;
@@ -128,8 +129,9 @@ __device__ void produce(const PipeArgs& a, unsigned char* stages, uint64_t* full
       info.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : p;
       info.is_last = t == end - 1;
       info.qs = q_scale_row(a.hp, t, b, t - s_indptr[b]);
-      // a unit with K or V heads needs the page id (unless K/V go to owned rows)
-      if (h0 + nh > a.hp.Hq && a.hp.out_k == nullptr)
+      // a unit with K or V heads, or of a last row (tail), needs the page id
+      // (unless K/V go to owned rows)
+      if ((h0 + nh > a.hp.Hq || info.is_last) && a.hp.out_k == nullptr)
         info.page = __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx);
       need_cs = (h0 < a.hp.Hq + a.hp.Hkv) && a.cs_bulk;
     }
@@ -233,6 +235,10 @@ __device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
+    // the request's last row: the block's consumer warps split its last-page
+    // tail (both caches) evenly, once per row (its first chunk)
+    if (info.is_last && c == 0 && a.hp.out_k == nullptr)
+      zero_tail_share(a.hp, info.page, info.slot_row, static_cast<uint32_t>(warp), a.wdiv, lane);
     if (++s == S) {
       s = 0;
       ph ^= 1u;
@@ -386,6 +392,7 @@ int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStr
   a.units = static_cast<int64_t>(p.T) * a.nchunks;
   if (a.units >= (int64_t{1} << 31)) return FQR_ENOTSUP;
   a.cdiv = FastDiv(static_cast<uint32_t>(a.nchunks));
+  a.wdiv = FastDiv(static_cast<uint32_t>(kConsumers));
   a.stage_bytes = stage_bytes(hc);
   // pipeline depth: aim at two resident blocks per SM (the register budget of
   // the consumers), never deeper than the units a block will see

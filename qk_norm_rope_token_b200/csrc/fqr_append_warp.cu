@@ -70,6 +70,33 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   const int gwarp = blockIdx.x * kWarps + warp;
   const int nwarps = gridDim.x * kWarps;
 
+  // While the preceding grid finishes: pull into L2 the lines of the first
+  // round trip below (metadata, weights, the first task's packed row and its
+  // own request's metadata), one prefetch per 128-byte line.
+  {
+    const int tid = threadIdx.x;
+    if (32 * tid <= a.B) {
+      prefetch_l2(a.q_indptr + 32 * tid);
+      if (32 * tid < a.B) prefetch_l2(a.seq_lens + 32 * tid);
+    }
+    const uint16_t* w = tid < 2 ? a.qw : a.kw;
+    if (tid < 4 && w != nullptr) prefetch_l2(w + 64 * (tid & 1));
+    if (gwarp < a.n_head) {
+      const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(gwarp)));
+      const int h = (gwarp - t * a.quads) * 4 + g;
+      if (l8 == 0 && h < a.H) {
+        const uint16_t* src = a.qkv + static_cast<int64_t>(t) * a.row_stride + h * kHeadDim;
+        prefetch_l2(src);
+        prefetch_l2(src + 64);
+      }
+      if (lane == 0) {
+        const int gb = t < a.B - 1 ? t : a.B - 1;
+        prefetch_l2(a.q_indptr + gb);
+        prefetch_l2(a.seq_lens + gb);
+        if (a.positions != nullptr) prefetch_l2(a.positions + t);
+      }
+    }
+  }
   grid_dependency_wait();
   grid_launch_dependents();
 
@@ -131,8 +158,7 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
       const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
       const int quad = w - t * a.quads;
       if (w == gwarp && early) {  // the batch is valid: the early lookups stand
-        process_quad_cs<POLICY, STYLE, false>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, s_w, l8,
-                                              gmask);
+        process_quad_cs<POLICY, STYLE>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, s_w, l8, gmask);
         if (paged && r0.is_last) zero_tail_share(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane);
         continue;
       }
@@ -152,8 +178,8 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
                    : 0;
       // (a group past the last head only helps with the tail)
       const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
-      process_quad<POLICY, STYLE, false, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, s_w, l8,
-                                                gmask);
+      process_quad<POLICY, STYLE, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, s_w, l8,
+                                         gmask);
       if (paged && r.is_last) zero_tail_share(a.hp, r.page, r.slot_row, quad, a.qdiv, lane);
     } else {
       const int b = w - a.n_head;  // request task: tail of a request without new rows

@@ -180,20 +180,6 @@ __device__ __forceinline__ void store_head(char* dst, const float2* y, int l8) {
   }
 }
 
-// Zero this head's column of the tail rows [row0 + 1, P) of a page: every
-// tail row is zeroed across its Hkv heads by the Hkv groups together.
-template <int ES>
-__device__ __forceinline__ void zero_tail_column(char* page_base, int row0, int P, int row_bytes,
-                                                 int kh, int l8) {
-  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-  char* col = page_base + static_cast<int64_t>(kh) * kHeadDim * ES + 16 * l8;
-  for (int row = row0 + 1; row < P; ++row) {
-    char* p = col + static_cast<int64_t>(row) * row_bytes;
-    st_v4(p, z);
-    if (ES == 2) st_v4(p + 128, z);
-  }
-}
-
 // A NeoX cos/sin row staged in shared memory is four 128-byte quarters
 // (cos 0-31, cos 32-63, sin 0-31, sin 32-63), each followed by 16 bytes of
 // padding: lane l8's 32-byte slice starts at quarter l8/4, byte 32*(l8%4),
@@ -268,16 +254,14 @@ __device__ __forceinline__ int quad_kind(const HeadParams& a, int h0) {
 // Norm + RoPE + quantisation + store of head h of row r.  xa/xb: the lane's two
 // 16-byte slices of the packed head; cs_row: the row's fp32 [cos | sin]
 // (shared or global memory); s_w: staged weights.  gmask: the 8-lane group.
-// TAILS: the K/V heads of a request's last row also zero their column of the
-// tail rows (when the caller does not split the tail over warps itself).
-// KIND: the head's kind when the caller knows it (HeadKind).
-template <int POLICY, int STYLE, bool TAILS = true, int KIND = kAnyHead>
+// KIND: the head's kind when the caller knows it (HeadKind).  Request tails
+// are zeroed by the callers (zero_tail_share), not here.
+template <int POLICY, int STYLE, int KIND = kAnyHead>
 __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCtx& r, int h,
                                                 uint4 xa, uint4 xb, const float2* c,
                                                 const float2* s, const float* s_w, int l8,
                                                 unsigned gmask) {
   constexpr int ES = POLICY == 0 ? 2 : 1;
-  const int P = a.page_size;
   float2 y[8];
   unpack_pairs(xa, xb, y);
 
@@ -295,8 +279,6 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
       divide_pairs(y, __ldg(a.v_scale));
       store_head<POLICY>(dst, y, l8);
     }
-    if (TAILS && r.is_last && a.out_v == nullptr)
-      zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
     return;
   }
 
@@ -378,26 +360,24 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
                     : page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
     if (POLICY != 0) divide_pairs(y, __ldg(a.k_scale));
     store_head<POLICY>(dst, y, l8);
-    if (TAILS && r.is_last && a.out_k == nullptr)
-      zero_tail_column<ES>(page_base, r.slot_row, P, a.row_bytes, kh, l8);
   }
 }
 
 // As process_head_cs, loading the cos/sin values from cs_row first (V heads
 // need none).
-template <int POLICY, int STYLE, bool CS_SMEM, bool TAILS = true, int KIND = kAnyHead>
+template <int POLICY, int STYLE, bool CS_SMEM, int KIND = kAnyHead>
 __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& r, int h,
                                              uint4 xa, uint4 xb, const float* cs_row,
                                              const float* s_w, int l8, unsigned gmask) {
   float2 c[4], s[4];
   if (KIND == kQHead || KIND == kKHead || (KIND == kAnyHead && h < a.Hq + a.Hkv))
     load_cs<STYLE, CS_SMEM>(cs_row, a.rot, l8, c, s);
-  process_head_cs<POLICY, STYLE, TAILS, KIND>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+  process_head_cs<POLICY, STYLE, KIND>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
 }
 
 // process_head_cs for one quad whose first head is h0 (warp-uniform), with
 // the cos/sin values already loaded; see process_quad.
-template <int POLICY, int STYLE, bool TAILS = true>
+template <int POLICY, int STYLE>
 __device__ __forceinline__ void process_quad_cs(const HeadParams& a, const RowCtx& r, int h0,
                                                 int nheads, int g, uint4 xa, uint4 xb,
                                                 const float2* c, const float2* s,
@@ -405,19 +385,19 @@ __device__ __forceinline__ void process_quad_cs(const HeadParams& a, const RowCt
   const int h = h0 + g;
   const int kind = h0 + 4 <= nheads ? quad_kind(a, h0) : kAnyHead;
   if (kind == kQHead)
-    process_head_cs<POLICY, STYLE, TAILS, kQHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+    process_head_cs<POLICY, STYLE, kQHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
   else if (kind == kKHead)
-    process_head_cs<POLICY, STYLE, TAILS, kKHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+    process_head_cs<POLICY, STYLE, kKHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
   else if (kind == kVHead)
-    process_head_cs<POLICY, STYLE, TAILS, kVHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+    process_head_cs<POLICY, STYLE, kVHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
   else if (h < nheads)
-    process_head_cs<POLICY, STYLE, TAILS, kAnyHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+    process_head_cs<POLICY, STYLE, kAnyHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
 }
 
 // process_head for one quad whose first head is h0 (warp-uniform): the kind
 // is decided once for the warp when all four heads exist; otherwise each
 // group decides for its own head (h0 + g < nheads).
-template <int POLICY, int STYLE, bool CS_SMEM, bool TAILS = true>
+template <int POLICY, int STYLE, bool CS_SMEM>
 __device__ __forceinline__ void process_quad(const HeadParams& a, const RowCtx& r, int h0,
                                              int nheads, int g, uint4 xa, uint4 xb,
                                              const float* cs_row, const float* s_w, int l8,
@@ -425,13 +405,13 @@ __device__ __forceinline__ void process_quad(const HeadParams& a, const RowCtx& 
   const int h = h0 + g;
   const int kind = h0 + 4 <= nheads ? quad_kind(a, h0) : kAnyHead;
   if (kind == kQHead)
-    process_head<POLICY, STYLE, CS_SMEM, TAILS, kQHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kQHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
   else if (kind == kKHead)
-    process_head<POLICY, STYLE, CS_SMEM, TAILS, kKHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kKHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
   else if (kind == kVHead)
-    process_head<POLICY, STYLE, CS_SMEM, TAILS, kVHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kVHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
   else if (h < nheads)
-    process_head<POLICY, STYLE, CS_SMEM, TAILS, kAnyHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kAnyHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
 }
 
 // Zero the whole tail (rows [last+1, P), all heads) of request b's last page in
