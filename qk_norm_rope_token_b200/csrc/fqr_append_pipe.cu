@@ -290,9 +290,29 @@ __global__ void __launch_bounds__(kPipeThreads, 2) pipe_append_kernel(const Pipe
     }
     mbar_init_fence();
   }
+  // While the preceding grid finishes: pull into L2 the metadata, the
+  // weights and the packed rows of this block's first two units, one
+  // prefetch per 128-byte line (L2 is the point of coherence: the reads after
+  // the wait still see the preceding grid's writes).
+  {
+    const int tid = threadIdx.x;
+    if (32 * tid <= a.B) {
+      prefetch_l2(a.q_indptr + 32 * tid);
+      if (32 * tid < a.B) prefetch_l2(a.seq_lens + 32 * tid);
+    }
+    const uint16_t* w = tid < 2 ? a.qw : a.kw;
+    if (tid < 4 && w != nullptr) prefetch_l2(w + 64 * (tid & 1));
+    for (int i = 0; i < 2 && i < nunits; ++i) {
+      int t, h0, nh;
+      unit_heads(a, u0 + i, t, h0, nh);
+      const uint16_t* src =
+          a.qkv + static_cast<int64_t>(t) * a.row_stride + static_cast<int64_t>(h0) * kHeadDim;
+      for (int l = tid; l < nh * 2; l += kPipeThreads) prefetch_l2(src + 64 * l);
+    }
+  }
   // Programmatic dependent launch: everything above touched only shared
-  // memory; wait for the preceding grid before reading any input, and let the
-  // next grid in the stream start its own set-up early.
+  // memory (and prefetched); wait for the preceding grid before reading any
+  // input, and let the next grid in the stream start its own set-up early.
   grid_dependency_wait();
   grid_launch_dependents();
   __syncthreads();

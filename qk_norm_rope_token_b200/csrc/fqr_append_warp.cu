@@ -70,6 +70,7 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   const int gwarp = blockIdx.x * kWarps + warp;
   const int nwarps = gridDim.x * kWarps;
 
+  const bool paged = a.hp.out_k == nullptr;
   // While the preceding grid finishes: pull into L2 the lines of the first
   // round trip below (metadata, weights, the first task's packed row and its
   // own request's metadata), one prefetch per 128-byte line.
@@ -89,11 +90,32 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
         prefetch_l2(src);
         prefetch_l2(src + 64);
       }
+      // ... and, from a possibly stale read of that metadata (L2 only), the
+      // lines of the second round trip: the page-table entry and the cos/sin
+      // row (a wrong guess costs only a useless prefetch)
+      const int gb = t < a.B - 1 ? t : a.B - 1;
+      int lo = 0, hi = 0, L = 0;
+      int64_t ps = 0;
       if (lane == 0) {
-        const int gb = t < a.B - 1 ? t : a.B - 1;
-        prefetch_l2(a.q_indptr + gb);
-        prefetch_l2(a.seq_lens + gb);
-        if (a.positions != nullptr) prefetch_l2(a.positions + t);
+        lo = ld_cg_s32(a.q_indptr + gb);
+        hi = ld_cg_s32(a.q_indptr + gb + 1);
+        L = ld_cg_s32(a.seq_lens + gb);
+        if (a.positions != nullptr) ps = ld_cg_s64(a.positions + t);
+      }
+      lo = __shfl_sync(0xffffffffu, lo, 0);
+      hi = __shfl_sync(0xffffffffu, hi, 0);
+      L = __shfl_sync(0xffffffffu, L, 0);
+      ps = __shfl_sync(0xffffffffu, ps, 0);
+      if (lo <= t && t < hi) {
+        const int p = t + L - hi;
+        const int64_t pos = a.positions != nullptr ? ps : static_cast<int64_t>(p);
+        if (p >= 0 && p < a.slot_cap && pos >= 0 && pos < a.cs_rows) {
+          if (lane == 0 && paged)
+            prefetch_l2(a.page_table + static_cast<int64_t>(gb) * a.max_pages +
+                        a.hp.pdiv.div(static_cast<uint32_t>(p)));
+          if (lane >= 1 && 32 * (lane - 1) < a.hp.rot && h < a.hp.Hq + a.hp.Hkv)
+            prefetch_l2(a.cs + pos * a.hp.rot + 32 * (lane - 1));
+        }
       }
     }
   }
@@ -106,7 +128,6 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   // row per request, the decode case).
   const MetaRegs meta = meta_prefetch(a.q_indptr, a.seq_lens, a.B);
   const float wreg = weight_prefetch(a.qw, a.kw, a.hp.gemma);
-  const bool paged = a.hp.out_k == nullptr;
   uint4 pa = make_uint4(0u, 0u, 0u, 0u), pb = pa;
   const bool head0 = gwarp < a.n_head;
   int t0 = 0, h0 = a.H, gb = 0, e_lo = 0, e_hi = 0, e_L = 0;

@@ -128,6 +128,29 @@ __device__ __forceinline__ void latent_row(const MlaArgs& a, int t, int b, int p
   }
 }
 
+// Before griddepcontrol.wait: pull into L2 the metadata lines and the inputs
+// of this warp's first task (latent row: kv_c and k_pe; Q quad: the rows of
+// its heads' rope part), one prefetch per 128-byte line.  L2 is the point of
+// coherence, so the reads after the wait still see the preceding grid's
+// writes.
+__device__ __forceinline__ void mla_prefetch(const MlaArgs& a, int64_t gwarp, int lane) {
+  const int tid = threadIdx.x;
+  if (32 * tid <= a.B) {
+    prefetch_l2(a.q_indptr + 32 * tid);
+    if (32 * tid < a.B) prefetch_l2(a.seq_lens + 32 * tid);
+  }
+  if (gwarp < a.T) {
+    const uint16_t* kc = a.kv_c + gwarp * a.kv_c_stride;
+    for (int l = lane; l < a.rank / 64; l += 32) prefetch_l2(kc + 64 * l);
+    if (lane == 0) prefetch_l2(a.k_pe + gwarp * a.k_pe_stride);
+  } else if (gwarp < a.T + static_cast<int64_t>(a.T) * a.qgroups && lane < 4) {
+    const int64_t qw = gwarp - a.T;
+    const int64_t t = qw / a.qgroups;
+    const int h = static_cast<int>(qw - t * a.qgroups) * 4 + lane;
+    if (h < a.Hq) prefetch_l2(a.q + t * a.q_tok + h * a.q_head + a.nope);
+  }
+}
+
 template <int FP8, int STYLE>
 __global__ void __launch_bounds__(kThreads) mla_kernel(const MlaArgs a) {
   extern __shared__ int smem[];
@@ -138,6 +161,7 @@ __global__ void __launch_bounds__(kThreads) mla_kernel(const MlaArgs a) {
   const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
 
+  mla_prefetch(a, gwarp, lane);
   grid_dependency_wait();
   grid_launch_dependents();
   const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
@@ -267,6 +291,7 @@ __global__ void __launch_bounds__(kThreads) mla_quant_kernel(const MlaArgs a) {
   const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
 
+  mla_prefetch(a, gwarp, lane);
   grid_dependency_wait();
   grid_launch_dependents();
   const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
@@ -329,6 +354,14 @@ __global__ void __launch_bounds__(kTokenWarps * 32) mla_token_kernel(const MlaAr
   const int gwarp = blockIdx.x * nw + warp;
   const int nwarps = gridDim.x * nw;
 
+  // before the wait: metadata, this warp's latent row and the block's first
+  // row of Q into L2 (see mla_prefetch)
+  mla_prefetch(a, gwarp < a.T ? gwarp : INT64_MAX, lane);
+  if (blockIdx.x < a.T) {
+    const uint16_t* qrow = a.q + static_cast<int64_t>(blockIdx.x) * a.q_tok;
+    const int64_t lines = (static_cast<int64_t>(a.Hq) * a.q_head + 63) / 64;
+    for (int64_t l = threadIdx.x; l < lines; l += blockDim.x) prefetch_l2(qrow + 64 * l);
+  }
   grid_dependency_wait();
   grid_launch_dependents();
   const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
