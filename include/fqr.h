@@ -45,7 +45,8 @@ extern "C" {
  * are identical).  AUTO picks LATENCY while every warp task of it (one per
  * 4 heads of a row, plus one per request) has a resident warp of its own --
  * small batches such as decode -- and STREAMING beyond that (large decode
- * batches, prefill). */
+ * batches, prefill); decode-like batches with large last-page tails (48 KiB
+ * or more expected per row) keep LATENCY up to 8 passes of tasks. */
 #define FQR_SCHEDULE_AUTO 0
 #define FQR_SCHEDULE_LATENCY 1
 #define FQR_SCHEDULE_STREAMING 2

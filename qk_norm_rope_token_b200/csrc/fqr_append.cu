@@ -13,6 +13,9 @@
 
 namespace fqr {
 
+constexpr int64_t kLargeTail = 48 * 1024;  // expected tail bytes per row (both caches)
+constexpr int64_t kLargeTailPasses = 8;
+
 int launch_append(const fqr_append_params& p, cudaStream_t stream) {
   HeadParams hp;
   const int es = p.quant_policy == 0 ? 2 : 1;
@@ -47,12 +50,24 @@ int launch_append(const fqr_append_params& p, cudaStream_t stream) {
 
   int schedule = p.schedule;
   if (schedule == FQR_SCHEDULE_AUTO) {
-    // latency while every warp task has a resident warp of its own (one
-    // pass, no task waits for another); streaming once the tasks outnumber
-    // the resident warps and a pipeline hides the rest
+    // Latency while every warp task has a resident warp of its own (one pass,
+    // no task waits for another); streaming once the tasks outnumber the
+    // resident warps and a pipeline hides the rest -- except for decode-like
+    // batches (a row per request) whose last-page tails are large (an
+    // expected kLargeTail bytes or more per row, half a page of both caches):
+    // the latency schedule writes those with bulk copies while its warps move
+    // on, and stays ahead up to kLargeTailPasses passes of tasks (measured on
+    // B200 with 64 FP8 Q heads, 8 KV heads and 64-slot pages).
     const int64_t cap = latency_capacity(p);
     if (cap < 0) return FQR_ECUDA;
-    schedule = latency_tasks(p) <= cap ? FQR_SCHEDULE_LATENCY : FQR_SCHEDULE_STREAMING;
+    const int64_t tasks = latency_tasks(p);
+    const int64_t tail_per_row =
+        owned ? 0 : static_cast<int64_t>(p.page_size - 1) * hp.row_bytes;  // (P-1)/2 rows x 2 caches
+    const bool decode_like = p.T <= p.B;
+    schedule = tasks <= cap || (decode_like && tail_per_row >= kLargeTail &&
+                                tasks <= kLargeTailPasses * cap)
+                   ? FQR_SCHEDULE_LATENCY
+                   : FQR_SCHEDULE_STREAMING;
   }
   return schedule == FQR_SCHEDULE_STREAMING ? launch_append_pipe(p, hp, stream)
                                             : launch_append_warp(p, hp, stream);

@@ -16,8 +16,9 @@
 //     whole batch (stage_and_validate); a malformed batch writes only flags.
 //   * the warps of a request's last new row split that request's last-page
 //     tail (both caches) evenly between them and store their share of zeros
-//     after their heads; one "request task" per request zeroes the tail of
-//     requests that append nothing.
+//     before their heads (the stores drain while the heads are computed);
+//     one "request task" per request zeroes the tail of requests that append
+//     nothing.
 #include "fqr_head.cuh"
 #include "fqr_launch.h"
 
@@ -40,8 +41,15 @@ struct WarpArgs {
   int max_pages;
   int64_t slot_cap;  // max_pages * page_size; INT64_MAX with caller-owned K/V
   int max_seqlen;    // > 0: the dynamic-Q prefill check n_b <= max_seqlen
+  int bulk_tail;     // tails by bulk copies (warps with several tasks)
   int32_t* flags;
 };
+
+// Shared memory: fp32 weights [256], q_indptr [B + 1], seq_lens [B], then the
+// zero buffer of the bulk tails (16-byte aligned).
+__host__ __device__ __forceinline__ int warp_zero_offset(int B) {
+  return ((2 * kHeadDim + 2 * B + 1) * static_cast<int>(sizeof(int)) + 15) & ~15;
+}
 
 __device__ __forceinline__ void warp_load_head(const WarpArgs& a, int w, int g, int l8, uint4& xa,
                                                uint4& xb) {
@@ -60,6 +68,8 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   float* s_w = reinterpret_cast<float*>(smem);  // 256 fp32 weights
   int* s_indptr = smem + 2 * kHeadDim;          // B + 1
   int* s_seq = s_indptr + a.B + 1;              // B
+  unsigned char* s_zero =                       // kZeroBytes (bulk tails)
+      reinterpret_cast<unsigned char*>(smem) + warp_zero_offset(a.B);
 
   // (a shuffled warp index is known to the compiler to be warp-uniform, so
   // the task loop and the head-kind dispatch branch uniformly)
@@ -166,6 +176,8 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
     }
   }
   weight_store(s_w, wreg);
+  if (a.bulk_tail) zero_buffer_init(s_zero);  // (the prologue's barrier follows)
+  bool issued = false;                        // bulk copies in flight (lane 0)
 
   const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T,
                a.B,         a.slot_cap,  a.cs_rows,  a.max_seqlen};
@@ -179,8 +191,15 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
       const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
       const int quad = w - t * a.quads;
       if (w == gwarp && early) {  // the batch is valid: the early lookups stand
+        // (the tail stores need nothing from the head: issue them first so they
+        // drain while the head is computed)
+        if (paged && r0.is_last) {
+          if (a.bulk_tail)
+            issued |= zero_tail_share_bulk(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane, s_zero);
+          else
+            zero_tail_share(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane);
+        }
         process_quad_cs<POLICY, STYLE>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, s_w, l8, gmask);
-        if (paged && r0.is_last) zero_tail_share(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane);
         continue;
       }
       const int h = quad * 4 + g;
@@ -197,11 +216,16 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
       r.page = paged && (h >= a.hp.Hq || r.is_last)
                    ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx)
                    : 0;
+      if (paged && r.is_last) {
+        if (a.bulk_tail)
+          issued |= zero_tail_share_bulk(a.hp, r.page, r.slot_row, quad, a.qdiv, lane, s_zero);
+        else
+          zero_tail_share(a.hp, r.page, r.slot_row, quad, a.qdiv, lane);
+      }
       // (a group past the last head only helps with the tail)
       const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
       process_quad<POLICY, STYLE, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, s_w, l8,
                                          gmask);
-      if (paged && r.is_last) zero_tail_share(a.hp, r.page, r.slot_row, quad, a.qdiv, lane);
     } else {
       const int b = w - a.n_head;  // request task: tail of a request without new rows
       const int L = s_seq[b];
@@ -209,6 +233,7 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
         zero_request_tail<POLICY == 0 ? 2 : 1>(a.hp, a.page_table, a.max_pages, b, L, lane);
     }
   }
+  if (issued) bulk_wait_all();  // the zero buffer must outlive the copies
 }
 
 using WarpKernel = void (*)(const WarpArgs);
@@ -225,7 +250,7 @@ static WarpKernel select_warp(int policy, int style) {
 }
 
 static size_t warp_smem(const fqr_append_params& p) {
-  return static_cast<size_t>(2 * kHeadDim + 2 * p.B + 1) * sizeof(int);
+  return static_cast<size_t>(warp_zero_offset(p.B)) + kZeroBytes;
 }
 
 int64_t latency_tasks(const fqr_append_params& p) {
@@ -276,7 +301,11 @@ int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStr
   const size_t smem = warp_smem(p);
   WarpKernel k = select_warp(p.quant_policy, p.rope_style);
   return launch_persistent(reinterpret_cast<const void*>(k), n_head + p.B, smem, stream,
-                           [&](int grid) { return launch_pdl(k, grid, kThreads, smem, stream, a); });
+                           [&](int grid) {
+                             // bulk tails once warps have more than one task
+                             a.bulk_tail = static_cast<int64_t>(grid) * kWarps < n_head + p.B;
+                             return launch_pdl(k, grid, kThreads, smem, stream, a);
+                           });
 }
 
 }  // namespace fqr

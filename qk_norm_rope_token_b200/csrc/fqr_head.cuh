@@ -237,6 +237,45 @@ __device__ __forceinline__ void zero_tail_share(const HeadParams& a, int page, i
   }
 }
 
+// The same share written by the TMA engine: lane 0 issues bulk copies from a
+// block-wide buffer of kZeroBytes zero bytes in shared memory (filled, and
+// fenced for the async proxy, before the block's first barrier) and commits
+// them as one bulk async-group; the issuing thread must bulk_wait_all()
+// before the block exits.  Returns whether this thread issued any copy.
+// The warp is then free for its next task while the zeros stream out, which
+// pays off when a warp has several tasks or large shares.
+constexpr uint32_t kZeroBytes = 2048;
+__device__ __forceinline__ bool zero_tail_share_bulk(const HeadParams& a, int page, int last,
+                                                     uint32_t part, const FastDiv& pdiv, int lane,
+                                                     const void* zbuf) {
+  const uint32_t span = static_cast<uint32_t>(a.page_size - 1 - last) * a.row_bytes;
+  const uint32_t units = span / 8;
+  const uint32_t u0 = pdiv.div(units * part), u1 = pdiv.div(units * (part + 1));
+  if (lane != 0 || u1 <= u0) return false;
+  const uint32_t o0 = u0 * 16, o1 = u1 * 16;  // byte range of [K span | V span]
+  const int64_t beg = static_cast<int64_t>(last + 1) * a.row_bytes;
+  char* kb = a.k_cache + static_cast<int64_t>(page) * a.k_page_bytes + beg;
+  char* vb = a.v_cache + static_cast<int64_t>(page) * a.v_page_bytes + beg;
+  if (o0 < span) {
+    const uint32_t e = o1 < span ? o1 : span;
+    for (uint32_t x = o0; x < e; x += kZeroBytes) bulk_s2g(kb + x, zbuf, min(kZeroBytes, e - x));
+  }
+  if (o1 > span) {
+    const uint32_t b = (o0 > span ? o0 : span) - span, e = o1 - span;
+    for (uint32_t x = b; x < e; x += kZeroBytes) bulk_s2g(vb + x, zbuf, min(kZeroBytes, e - x));
+  }
+  bulk_commit();
+  return true;
+}
+
+// Fill the block's zero buffer (kZeroBytes, 16-byte aligned) and order the
+// writes before the bulk copies that read it; a block barrier must follow.
+__device__ __forceinline__ void zero_buffer_init(unsigned char* zbuf) {
+  for (uint32_t i = threadIdx.x; i < kZeroBytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(zbuf)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+}
+
 // What the 4 heads of a quad are, when the whole quad is known to be of one
 // kind (a warp-uniform value, so the per-head code has no divergent branch
 // on the head type); kAnyHead decides per head.
