@@ -133,21 +133,51 @@ __device__ __forceinline__ void latent_row(const MlaArgs& a, int t, int b, int p
 // its heads' rope part), one prefetch per 128-byte line.  L2 is the point of
 // coherence, so the reads after the wait still see the preceding grid's
 // writes.
+// Then, from a possibly stale read of the task's own request metadata (L2
+// only: the values only steer prefetches, and a later load cannot hit a
+// stale L1 line; the request is guessed as b = t, one row per request), the
+// block-table entry and the cos/sin row of that row.
 __device__ __forceinline__ void mla_prefetch(const MlaArgs& a, int64_t gwarp, int lane) {
   const int tid = threadIdx.x;
   if (32 * tid <= a.B) {
     prefetch_l2(a.q_indptr + 32 * tid);
     if (32 * tid < a.B) prefetch_l2(a.seq_lens + 32 * tid);
   }
+  int64_t t = -1;
   if (gwarp < a.T) {
+    t = gwarp;
     const uint16_t* kc = a.kv_c + gwarp * a.kv_c_stride;
     for (int l = lane; l < a.rank / 64; l += 32) prefetch_l2(kc + 64 * l);
     if (lane == 0) prefetch_l2(a.k_pe + gwarp * a.k_pe_stride);
-  } else if (gwarp < a.T + static_cast<int64_t>(a.T) * a.qgroups && lane < 4) {
+  } else if (gwarp < a.T + static_cast<int64_t>(a.T) * a.qgroups) {
     const int64_t qw = gwarp - a.T;
-    const int64_t t = qw / a.qgroups;
+    t = qw / a.qgroups;
     const int h = static_cast<int>(qw - t * a.qgroups) * 4 + lane;
-    if (h < a.Hq) prefetch_l2(a.q + t * a.q_tok + h * a.q_head + a.nope);
+    if (lane < 4 && h < a.Hq) prefetch_l2(a.q + t * a.q_tok + h * a.q_head + a.nope);
+  }
+  if (t < 0) return;  // (warp-uniform)
+  const int gb = t < a.B - 1 ? static_cast<int>(t) : a.B - 1;
+  int lo = 0, hi = 0, L = 0;
+  int64_t ps = 0;
+  if (lane == 0) {
+    lo = ld_cg_s32(a.q_indptr + gb);
+    hi = ld_cg_s32(a.q_indptr + gb + 1);
+    L = ld_cg_s32(a.seq_lens + gb);
+    if (a.positions != nullptr) ps = ld_cg_s64(a.positions + t);
+  }
+  lo = __shfl_sync(0xffffffffu, lo, 0);
+  hi = __shfl_sync(0xffffffffu, hi, 0);
+  L = __shfl_sync(0xffffffffu, L, 0);
+  ps = __shfl_sync(0xffffffffu, ps, 0);
+  if (lo <= t && t < hi) {
+    const int64_t p = t + L - hi;
+    const int64_t pos = a.positions != nullptr ? ps : p;
+    if (p >= 0 && p < static_cast<int64_t>(a.max_blocks) * a.block_size && pos >= 0 &&
+        pos < a.cs_rows) {
+      if (lane == 0 && gwarp < a.T)
+        prefetch_l2(a.block_table + static_cast<int64_t>(gb) * a.max_blocks + p / a.block_size);
+      if (lane == 1 || lane == 2) prefetch_l2(a.cs + pos * kRope + 32 * (lane - 1));
+    }
   }
 }
 
