@@ -18,7 +18,8 @@ launch / average launch time, against the measured HBM copy bandwidth;
 `e2e` = the same metric through the public API with pinned host buffers
 (host->device copies of the step's inputs and device->host copies of out_q
 and flags inside the timed region); `cpu_baseline` = the CPU oracle on a
-bounded sample; `per_config` adds the other named workloads (kernel time,
+bounded sample, single-threaded (`cpu_baseline_all_cores`: one process per
+host core on disjoint requests); `per_config` adds the other named workloads (kernel time,
 GB/s, fraction of peak) measured the same way, outside the timed region.
 
 --impl reference times the CPU oracle (the reference arm of this build) on
@@ -453,46 +454,92 @@ def cpu_baseline(w, budget_s):
                       f"{el:.1f} s single-threaded C oracle (fp32, -O2, no FMA)"}
 
 
+def _oracle_worker(job):
+    """One process of the all-cores baseline: whole calls of a sub-batch."""
+    w, budget_s = job
+    calls, el = oracle_sample(w, budget_s)
+    return w.T * calls, el
+
+
+def cpu_baseline_all_cores(w, budget_s, cores=None):
+    """The oracle as it stands, one process per host core, each on its own
+    whole requests of the workload (disjoint sub-batches are valid calls of
+    their own) for budget_s seconds; throughput = all tokens / the longest
+    worker's time.  Processes are spawned (never forked after CUDA use)."""
+    import multiprocessing as mp
+    n = max(1, min(cores or os.cpu_count() or 1, w.B))
+    per = -(-w.B // n)
+    subs = [_sub_batch(w, b0, min(w.B, b0 + per)) for b0 in range(0, w.B, per)]
+    with mp.get_context("spawn").Pool(len(subs)) as pool:
+        res = pool.map(_oracle_worker, [(sb, budget_s) for sb in subs])
+    tokens = sum(r[0] for r in res)
+    el = max(r[1] for r in res)
+    return {"value": tokens / el, "unit": UNIT, "cores": len(subs), "kind": "oracle",
+            "sample": f"{len(subs)} processes, each whole calls of {per} requests of {w.name} "
+                      f"for {budget_s:.0f} s ({tokens} tokens in all); single-threaded C oracle "
+                      f"per process (fp32, -O2, no FMA)"}
+
+
+def _reference_worker(job):
+    """One process of the reference arm: W warm-up and K timed steps, each
+    one whole oracle call over the next of this worker's sub-batches."""
+    subs, warmup, steps = job
+    import oracle
+    w = subs[0]
+    dt = np.uint16 if w.kv_esize == 2 else np.uint8
+    kc = np.zeros((w.num_pages, w.page_size, w.Hkv, 128), dt)
+    vc = np.zeros_like(kc)
+    outs = [oracle.new_outputs(sb) for sb in subs]
+
+    def step(i):
+        sb = subs[i % len(subs)]
+        oq, qs, fl = outs[i % len(subs)]
+        assert oracle.append_paged(sb, kc, vc, oq, qs if sb.quant_policy == 1 else None, fl) == 0
+        return sb.T
+
+    for i in range(warmup):
+        step(i)
+    t0 = time.perf_counter()
+    toks = sum(step(i) for i in range(steps))
+    return toks, time.perf_counter() - t0
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
     w = workloads.APPEND_CONFIGS[args.workload]()
-    import oracle
-    # size each step's sample so the whole run stays within a few minutes
+    # the oracle as it stands on the host cores: one spawned process per core,
+    # each on its own whole requests; every step, each process runs one call
+    # over a sample of its requests, sized so the whole run stays within a
+    # few minutes
+    n = max(1, min(os.cpu_count() or 1, w.B))
     calls, el = oracle_sample(w, 0.0, max_calls=2)
-    t_call = el / calls
-    per_token = t_call / max(w.T, 1)
+    per_token = el / calls / max(w.T, 1)
     budget = 120.0
-    tokens = int(max(1, min(w.T, budget / max(1, args.steps + args.warmup) / per_token)))
-    subs = []
-    for b0 in range(0, w.B, tokens):
-        subs.append(_sub_batch(w, b0, min(w.B, b0 + tokens)))
-    es = w.kv_esize
-    dt = np.uint16 if es == 2 else np.uint8
-    kc = np.zeros((w.num_pages, w.page_size, w.Hkv, 128), dt)
-    vc = np.zeros_like(kc)
-    outs = [oracle.new_outputs(s) for s in subs]
-
-    def step(i):
-        s = subs[i % len(subs)]
-        oq, qs, fl = outs[i % len(subs)]
-        assert oracle.append_paged(s, kc, vc, oq, qs if s.quant_policy == 1 else None, fl) == 0
-        return s.T
-
-    for i in range(args.warmup):
-        step(i)
-    t0 = time.perf_counter()
-    toks = sum(step(i) for i in range(args.steps))
-    el = time.perf_counter() - t0
+    per_worker = -(-w.B // n)
+    tokens = int(max(1, min(per_worker, budget / max(1, args.steps + args.warmup) / per_token)))
+    jobs = []
+    for j in range(n):
+        lo, hi = j * per_worker, min(w.B, (j + 1) * per_worker)
+        if lo >= hi:
+            break
+        subs = [_sub_batch(w, b0, min(hi, b0 + tokens)) for b0 in range(lo, hi, tokens)]
+        jobs.append((subs, args.warmup, args.steps))
+    import multiprocessing as mp
+    with mp.get_context("spawn").Pool(len(jobs)) as pool:
+        res = pool.map(_reference_worker, jobs)
+    toks = sum(r[0] for r in res)
+    el = max(r[1] for r in res)
     value = toks / el
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "config": config_block(w, None),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{args.steps} steps of {tokens} request(s) x 1 token of "
-                                   f"{w.name}, single-threaded C oracle"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": len(jobs), "kind": "oracle",
+                         "sample": f"{len(jobs)} processes x {args.steps} steps, each step one "
+                                   f"call over {tokens} request(s) of the process's own share of "
+                                   f"{w.name}; single-threaded C oracle per process"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -584,9 +631,10 @@ def main(argv=None):
     per_config = None
     if rank == 0 and not args.no_per_config:
         per_config = measure_per_config(torch, fqr, dev, peak, args.workload)
-    cpu = None
+    cpu = cpu_all = None
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         cpu = cpu_baseline(bench.ws[0], args.cpu_seconds)
+        cpu_all = cpu_baseline_all_cores(bench.ws[0], args.cpu_seconds)
     if dist is not None:
         barrier()
         dist.destroy_process_group()
@@ -601,9 +649,11 @@ def main(argv=None):
                      "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
                      "peak_source": peak_src,
                      "bytes_per_launch": nbytes / args.steps,
-                     "kernel": "fqr::append_kernel", "timing": "CUDA events around graph "
+                     "kernel": "fqr::warp_append_kernel<0,0> (latency schedule, chosen "
+                     "automatically)", "timing": "CUDA events around graph "
                      "replays of back-to-back launches; average launch = region / steps"},
         "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks, "cpu_baseline": cpu,
+        "cpu_baseline_all_cores": cpu_all,
         "per_config": per_config,
     }
     print(json.dumps(line), flush=True)
