@@ -81,6 +81,19 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   const int nwarps = gridDim.x * kWarps;
 
   const bool paged = a.hp.out_k == nullptr;
+  // The first task's coordinates need only the kernel parameters: computed
+  // once, for the prefetches below and for the loads after the wait.
+  const bool head0 = gwarp < a.n_head;
+  int t0 = 0, h0 = a.H, gb = 0;
+  const uint16_t* src0 = a.qkv;
+  if (head0) {
+    t0 = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(gwarp)));
+    h0 = (gwarp - t0 * a.quads) * 4 + g;
+    gb = t0 < a.B - 1 ? t0 : a.B - 1;
+    src0 = a.qkv + static_cast<int64_t>(t0) * a.row_stride + h0 * kHeadDim + 8 * l8;
+  }
+  const bool own0 = head0 && h0 < a.H;  // this group has a head in the first task
+
   // While the preceding grid finishes: pull into L2 the lines of the first
   // round trip below (metadata, weights, the first task's packed row and its
   // own request's metadata), one prefetch per 128-byte line.
@@ -92,38 +105,34 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
     }
     const uint16_t* w = tid < 2 ? a.qw : a.kw;
     if (tid < 4 && w != nullptr) prefetch_l2(w + 64 * (tid & 1));
-    if (gwarp < a.n_head) {
-      const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(gwarp)));
-      const int h = (gwarp - t * a.quads) * 4 + g;
-      if (l8 == 0 && h < a.H) {
-        const uint16_t* src = a.qkv + static_cast<int64_t>(t) * a.row_stride + h * kHeadDim;
-        prefetch_l2(src);
-        prefetch_l2(src + 64);
+    if (head0) {
+      if (l8 == 0 && own0) {
+        prefetch_l2(src0);
+        prefetch_l2(src0 + 64);
       }
       // ... and, from a possibly stale read of that metadata (L2 only), the
       // lines of the second round trip: the page-table entry and the cos/sin
       // row (a wrong guess costs only a useless prefetch)
-      const int gb = t < a.B - 1 ? t : a.B - 1;
       int lo = 0, hi = 0, L = 0;
       int64_t ps = 0;
       if (lane == 0) {
         lo = ld_cg_s32(a.q_indptr + gb);
         hi = ld_cg_s32(a.q_indptr + gb + 1);
         L = ld_cg_s32(a.seq_lens + gb);
-        if (a.positions != nullptr) ps = ld_cg_s64(a.positions + t);
+        if (a.positions != nullptr) ps = ld_cg_s64(a.positions + t0);
       }
       lo = __shfl_sync(0xffffffffu, lo, 0);
       hi = __shfl_sync(0xffffffffu, hi, 0);
       L = __shfl_sync(0xffffffffu, L, 0);
       ps = __shfl_sync(0xffffffffu, ps, 0);
-      if (lo <= t && t < hi) {
-        const int p = t + L - hi;
+      if (lo <= t0 && t0 < hi) {
+        const int p = t0 + L - hi;
         const int64_t pos = a.positions != nullptr ? ps : static_cast<int64_t>(p);
         if (p >= 0 && p < a.slot_cap && pos >= 0 && pos < a.cs_rows) {
           if (lane == 0 && paged)
             prefetch_l2(a.page_table + static_cast<int64_t>(gb) * a.max_pages +
                         a.hp.pdiv.div(static_cast<uint32_t>(p)));
-          if (lane >= 1 && 32 * (lane - 1) < a.hp.rot && h < a.hp.Hq + a.hp.Hkv)
+          if (lane >= 1 && 32 * (lane - 1) < a.hp.rot && h0 < a.hp.Hq + a.hp.Hkv)
             prefetch_l2(a.cs + pos * a.hp.rot + 32 * (lane - 1));
         }
       }
@@ -139,14 +148,13 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   const MetaRegs meta = meta_prefetch(a.q_indptr, a.seq_lens, a.B);
   const float wreg = weight_prefetch(a.qw, a.kw, a.hp.gemma);
   uint4 pa = make_uint4(0u, 0u, 0u, 0u), pb = pa;
-  const bool head0 = gwarp < a.n_head;
-  int t0 = 0, h0 = a.H, gb = 0, e_lo = 0, e_hi = 0, e_L = 0;
+  int e_lo = 0, e_hi = 0, e_L = 0;
   int64_t e_pos = 0;
   if (head0) {
-    t0 = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(gwarp)));
-    h0 = (gwarp - t0 * a.quads) * 4 + g;
-    warp_load_head(a, gwarp, g, l8, pa, pb);
-    gb = t0 < a.B - 1 ? t0 : a.B - 1;
+    if (own0) {
+      pa = ld_stream_v4(src0);
+      pb = ld_stream_v4(src0 + 64);
+    }
     e_lo = __ldg(a.q_indptr + gb);
     e_hi = __ldg(a.q_indptr + gb + 1);
     e_L = __ldg(a.seq_lens + gb);
