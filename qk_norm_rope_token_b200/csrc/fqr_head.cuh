@@ -145,25 +145,26 @@ __device__ __forceinline__ float2 div2_bounded(float2 a, float2 b, float2 r) {
 }
 
 // K / V payloads: every value divided by d (k_scale or v_scale, one value for
-// the whole call), then encoded to E4M3.  The lane's 16 quotients come from
+// the whole call), then encoded to E4M3.  The lane's 2N quotients come from
 // div2_bounded when the division cannot overflow or lose the exactness of the
 // residual anywhere it matters -- 2^-80 <= d <= 2^80 and max|x| / d < 2^100
 // -- which makes every E4M3 code equal to the code of the IEEE quotient
 // (tests/test_gpu_division.py checks it over every binary32 dividend for a set
 // of scales).  A negative scale would give a zero quotient the wrong sign in
 // the correction; it, like any lane outside the guard, divides with __fdiv_rn.
+template <int N = 8>
 __device__ __forceinline__ void divide_pairs(float2* y, float d) {
   const float r = __frcp_rn(d);
   float m = 0.0f;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) m = fmaxf(m, fmaxf(fabsf(y[j].x), fabsf(y[j].y)));
+  for (int j = 0; j < N; ++j) m = fmaxf(m, fmaxf(fabsf(y[j].x), fabsf(y[j].y)));
   if (d >= 0x1p-80f && d <= 0x1p80f && m * r < 0x1p100f) {
     const float2 b2 = make_float2(d, d), r2 = make_float2(r, r);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = div2_bounded(y[j], b2, r2);
+    for (int j = 0; j < N; ++j) y[j] = div2_bounded(y[j], b2, r2);
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = make_float2(__fdiv_rn(y[j].x, d), __fdiv_rn(y[j].y, d));
+    for (int j = 0; j < N; ++j) y[j] = make_float2(__fdiv_rn(y[j].x, d), __fdiv_rn(y[j].y, d));
   }
 }
 

@@ -86,39 +86,79 @@ __device__ __forceinline__ void mla_rotate(float* y /* A[0..4) B[4..8) */, const
   }
 }
 
-// Latent row of packed row t (request b, slot position p_slot): 32 lanes
-// encode kv_c in 16-byte vectors, 8 lanes rotate k_pe.
+// E4M3 latent payloads x / kv_scale for 8 values: the guarded Markstein
+// division of fqr_head.cuh (divide_pairs: codes equal to IEEE division's).
+__device__ __forceinline__ void divide8(float* y, float d) {
+  float2 v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) v[j] = make_float2(y[2 * j], y[2 * j + 1]);
+  divide_pairs<4>(v, d);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    y[2 * j] = v[j].x;
+    y[2 * j + 1] = v[j].y;
+  }
+}
+
+// A latent row's inputs as one lane holds them: kv_c chunks lane + 32 k
+// (8 elements each; kLatentChunks in registers, any further ones are loaded
+// when stored) and, for lanes < 8, the k_pe elements [4l, 4l+4) and
+// [32+4l, 32+4l+4).
+constexpr int kLatentChunks = 2;  // kv_lora_rank 512
+struct LatentIn {
+  uint4 kv[kLatentChunks];
+  uint2 pe0, pe1;
+};
+
+__device__ __forceinline__ void load_latent(const MlaArgs& a, int t, int lane, LatentIn& in) {
+  const uint16_t* kc = a.kv_c + static_cast<int64_t>(t) * a.kv_c_stride;
+#pragma unroll
+  for (int k = 0; k < kLatentChunks; ++k)
+    if (lane + 32 * k < a.rank / 8) in.kv[k] = ld_stream_v4(kc + 8 * (lane + 32 * k));
+  if (lane < kRope / 8) {
+    const uint16_t* kp = a.k_pe + static_cast<int64_t>(t) * a.k_pe_stride;
+    in.pe0 = ld_stream_v2(kp + 4 * lane);
+    in.pe1 = ld_stream_v2(kp + kRope / 2 + 4 * lane);
+  }
+}
+
+// Latent row of packed row t (request b, slot position p_slot) from `in`:
+// the encoded row goes to its block slot.
 template <int FP8, int STYLE>
-__device__ __forceinline__ void latent_row(const MlaArgs& a, int t, int b, int p_slot,
-                                           const float* row, int lane) {
+__device__ __forceinline__ void store_latent(const MlaArgs& a, int t, int b, int p_slot,
+                                             const float* row, int lane, const LatentIn& in) {
   const int64_t blk =
       __ldg(a.block_table + static_cast<int64_t>(b) * a.max_blocks + p_slot / a.block_size);
   char* dst = a.latent + (blk * a.block_size + p_slot % a.block_size) * a.row_bytes;
   const uint16_t* kc = a.kv_c + static_cast<int64_t>(t) * a.kv_c_stride;
   const float sc = FP8 ? __ldg(a.kv_scale) : 1.0f;
-  for (int c8 = lane; c8 < a.rank / 8; c8 += 32) {
-    const uint4 v = ld_stream_v4(kc + 8 * c8);
+  for (int k = 0, c8 = lane; c8 < a.rank / 8; ++k, c8 += 32) {
+    uint4 v;
+    if (k < kLatentChunks) {
+#pragma unroll
+      for (int j = 0; j < kLatentChunks; ++j)
+        if (j == k) v = in.kv[j];
+    } else {
+      v = ld_stream_v4(kc + 8 * c8);
+    }
     if (FP8) {
       float y[8];
       unpack8(v, y);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) y[k] = __fdiv_rn(y[k], sc);
+      divide8(y, sc);
       st_v2(dst + 8 * c8, pack8_e4m3(y));
     } else {
       st_v4(dst + 16 * c8, v);
     }
   }
   if (lane < kRope / 8) {
-    const uint16_t* kp = a.k_pe + static_cast<int64_t>(t) * a.k_pe_stride;
     float y[8], c[4], s[4];
-    unpack4(ld_stream_v2(kp + 4 * lane), y);
-    unpack4(ld_stream_v2(kp + kRope / 2 + 4 * lane), y + 4);
+    unpack4(in.pe0, y);
+    unpack4(in.pe1, y + 4);
     mla_cos_sin<STYLE>(row, lane, c, s);
     mla_rotate<STYLE>(y, c, s);
     const int64_t e0 = a.rank + 4 * lane, e1 = a.rank + kRope / 2 + 4 * lane;
     if (FP8) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) y[k] = __fdiv_rn(y[k], sc);
+      divide8(y, sc);
       st_u32(dst + e0, pack4_e4m3(y));
       st_u32(dst + e1, pack4_e4m3(y + 4));
     } else {
@@ -126,6 +166,14 @@ __device__ __forceinline__ void latent_row(const MlaArgs& a, int t, int b, int p
       st_v2(dst + 2 * e1, pack4_bf16(y + 4));
     }
   }
+}
+
+template <int FP8, int STYLE>
+__device__ __forceinline__ void latent_row(const MlaArgs& a, int t, int b, int p_slot,
+                                           const float* row, int lane) {
+  LatentIn in;
+  load_latent(a, t, lane, in);
+  store_latent<FP8, STYLE>(a, t, b, p_slot, row, lane, in);
 }
 
 // Before griddepcontrol.wait: pull into L2 the metadata lines and the inputs
@@ -194,12 +242,30 @@ __global__ void __launch_bounds__(kThreads) mla_kernel(const MlaArgs a) {
   mla_prefetch(a, gwarp, lane);
   grid_dependency_wait();
   grid_launch_dependents();
+
+  // the first task's inputs need no metadata: load them before the
+  // validation prologue (a latent row, or this group's head of a Q quad)
+  const int64_t n_lat = a.T;
+  const int64_t n_tasks = n_lat + static_cast<int64_t>(a.T) * a.qgroups;
+  LatentIn in0;
+  uint2 q0a = make_uint2(0u, 0u), q0b = q0a;
+  if (gwarp < n_lat) {
+    load_latent(a, static_cast<int>(gwarp), lane, in0);
+  } else if (gwarp < n_tasks) {
+    const int64_t qw = gwarp - n_lat;
+    const int64_t t = qw / a.qgroups;
+    const int h = static_cast<int>(qw - t * a.qgroups) * 4 + g;
+    if (h < a.Hq) {
+      const uint16_t* qp = a.q + t * a.q_tok + h * a.q_head + a.nope;
+      q0a = ld_v2(qp + 4 * l8);
+      q0b = ld_v2(qp + kRope / 2 + 4 * l8);
+    }
+  }
+
   const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
                static_cast<int64_t>(a.max_blocks) * a.block_size, a.cs_rows};
   if (stage_and_validate(m, s_indptr, s_seq)) return;
 
-  const int64_t n_lat = a.T;
-  const int64_t n_tasks = n_lat + static_cast<int64_t>(a.T) * a.qgroups;
   for (int64_t w = gwarp; w < n_tasks; w += nwarps) {
     const bool lat = w < n_lat;
     const int64_t qw = w - n_lat;
@@ -210,14 +276,17 @@ __global__ void __launch_bounds__(kThreads) mla_kernel(const MlaArgs a) {
     const float* row = a.cs + pos * kRope;
 
     if (lat) {
-      latent_row<FP8, STYLE>(a, t, b, p_slot, row, lane);
+      if (w == gwarp)
+        store_latent<FP8, STYLE>(a, t, b, p_slot, row, lane, in0);
+      else
+        latent_row<FP8, STYLE>(a, t, b, p_slot, row, lane);
     } else {
       const int h = static_cast<int>(qw - static_cast<int64_t>(t) * a.qgroups) * 4 + g;
       if (h < a.Hq) {
         uint16_t* qp = a.q + static_cast<int64_t>(t) * a.q_tok + h * a.q_head + a.nope;
         float y[8], c[4], s[4];
-        unpack4(ld_v2(qp + 4 * l8), y);
-        unpack4(ld_v2(qp + kRope / 2 + 4 * l8), y + 4);
+        unpack4(w == gwarp ? q0a : ld_v2(qp + 4 * l8), y);
+        unpack4(w == gwarp ? q0b : ld_v2(qp + kRope / 2 + 4 * l8), y + 4);
         mla_cos_sin<STYLE>(row, l8, c, s);
         mla_rotate<STYLE>(y, c, s);
         st_v2(qp + 4 * l8, pack4_bf16(y));
