@@ -377,51 +377,61 @@ def time_launches(torch, bench, steps, warmup, graph_chunk=1000, barrier=None, m
 
 
 def e2e_measure(torch, fqr, bench, steps):
-    """Same metric through the public API with pinned host buffers."""
+    """Same metric through the public API with pinned host buffers: every
+    step copies its inputs host->device, runs the kernel and copies out_q and
+    flags device->host (StagedAppend: copy-in of step i+1, kernel of step i
+    and copy-out of step i-1 overlap on three streams)."""
     w0 = bench.ws[0]
     dev = bench.dev
     R = min(bench.R, 8)
+    in_shapes = {"qkv": ((w0.T, w0.row_stride), torch.int16),
+                 "q_indptr": ((w0.B + 1,), torch.int32), "seq_lens": ((w0.B,), torch.int32),
+                 "page_table": (tuple(w0.page_table.shape), torch.int32)}
+    out_shapes = {"out_q": (tuple(bench.reps[0]["out_q"].shape), bench.reps[0]["out_q"].dtype),
+                  "flags": ((w0.B,), torch.int32)}
+    if w0.quant_policy == 1:
+        out_shapes["q_scale"] = ((w0.T, w0.Hq), torch.float32)
+    kw = bench.kw_for(w0, {"q_scale": None})
+    kw.pop("q_scale", None)
+    sa = fqr.StagedAppend(in_shapes, out_shapes, dev, depth=3, cos_sin_cache=bench.cs,
+                          k_cache=bench.k_cache, v_cache=bench.v_cache, **kw)
     host_in, host_out = [], []
     for w in bench.ws[:R]:
-        hi = {"qkv": torch.from_numpy(w.qkv.view(np.int16)).pin_memory(),
-              "q_indptr": torch.from_numpy(w.q_indptr).pin_memory(),
-              "seq_lens": torch.from_numpy(w.seq_lens).pin_memory(),
-              "page_table": torch.from_numpy(w.page_table).pin_memory()}
+        hi, ho = sa.new_host_buffers()
+        hi["qkv"].copy_(torch.from_numpy(w.qkv.view(np.int16)))
+        hi["q_indptr"].copy_(torch.from_numpy(w.q_indptr))
+        hi["seq_lens"].copy_(torch.from_numpy(w.seq_lens))
+        hi["page_table"].copy_(torch.from_numpy(w.page_table))
         host_in.append(hi)
-        ho = {"out_q": torch.empty(bench.reps[0]["out_q"].shape,
-                                   dtype=bench.reps[0]["out_q"].dtype).pin_memory(),
-              "flags": torch.empty((w.B,), dtype=torch.int32).pin_memory()}
-        if w.quant_policy == 1:
-            ho["q_scale"] = torch.empty((w.T, w.Hq), dtype=torch.float32).pin_memory()
         host_out.append(ho)
-    dev_in = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in host_in[0].items()}
-    dev_out = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in host_out[0].items()}
-    kw = bench.kw_for(w0, {"q_scale": dev_out.get("q_scale")})
-    kw.pop("q_scale", None)
-    h2d = sum(v.numel() * v.element_size() for v in host_in[0].values())
-    d2h = sum(v.numel() * v.element_size() for v in host_out[0].values())
+    h2d = int(host_in[0]["_flat"].numel())
+    d2h = int(host_out[0]["_flat"].numel())
 
     def step(i):
-        fqr.append_paged_from_host(host_in[i % R], dev_in, host_out[i % R], dev_out,
-                                   cos_sin_cache=bench.cs, k_cache=bench.k_cache,
-                                   v_cache=bench.v_cache, **kw)
+        return sa.submit(host_in[i % R], host_out[i % R])
 
     for i in range(20):
         step(i)
+    sa.synchronize()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
+    for st in (sa.s_in, sa.s_k, sa.s_out):
+        st.wait_event(start)
+    last = None
     for i in range(steps):
-        step(i)
+        last = step(i)
+    stream.wait_event(last)   # the last copy-out follows every earlier step's work
     end.record(stream)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
     assert int(host_out[(steps - 1) % R]["flags"].abs().max()) == 0
-    return {"value": bench.T * steps / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "ms_per_step": ms / steps}
+    return {"value": bench.T * steps / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps,
+            "api": "qk_norm_rope_token_b200.StagedAppend (3 streams, 3 staging buffers, one "
+                   "flat pinned buffer each way)"}
 
 
 # ----------------------------------------------------------- CPU baselines

@@ -14,6 +14,8 @@ as torch.float8_e4m3fn or torch.uint8.  All on one CUDA device.
 from __future__ import annotations
 
 import ctypes
+
+import numpy as np
 import os
 from typing import Optional
 
@@ -192,6 +194,124 @@ def append_paged_from_host(host_in: dict, dev_in: dict, host_out: dict, dev_out:
             h.copy_(dev_out[k], non_blocking=True)
 
 
+class StagedAppend:
+    """append_paged on batches that live in pinned host memory, pipelined.
+
+    Each submit() enqueues, for one batch: the host-to-device copy of its
+    inputs on a copy-in stream, the fused kernel on a compute stream, and the
+    device-to-host copy of its results on a copy-out stream, with events
+    between them and `depth` sets of device staging buffers rotated.  So the
+    copy-in of the next batch, the kernel of this one and the copy-out of the
+    previous one overlap (PCIe carries both directions at once).
+
+    in_shapes / out_shapes map the names of append_paged_from_host ("qkv",
+    "q_indptr", "seq_lens", "page_table", optionally "positions"; "out_q",
+    "flags", optionally "q_scale") to (shape, dtype).  Each slot's inputs
+    (and results) are views of one flat device buffer, so host buffers made
+    by new_host_buffers() -- views of one flat pinned buffer -- move in one
+    copy each way.  The KV caches, cos/sin cache, norm weights and the other
+    append_paged keywords are fixed at construction (each slot's parameter
+    block is built once).  synchronize() waits for every submitted batch;
+    read a batch's host results after that, or after the event submit()
+    returns."""
+
+    _ALIGN = 256
+
+    def __init__(self, in_shapes: dict, out_shapes: dict, device, depth: int = 2, *,
+                 cos_sin_cache, k_cache, v_cache, **kw):
+        import torch
+        self.torch = torch
+        self.depth = depth
+        self.in_shapes, self.out_shapes = dict(in_shapes), dict(out_shapes)
+        self.in_bytes, self.in_offs = self._layout(self.in_shapes)
+        self.out_bytes, self.out_offs = self._layout(self.out_shapes)
+        self.flat_in = [torch.empty(self.in_bytes, dtype=torch.uint8, device=device) for _ in range(depth)]
+        self.flat_out = [torch.empty(self.out_bytes, dtype=torch.uint8, device=device)
+                         for _ in range(depth)]
+        self.dev_in = [self._views(f, self.in_shapes, self.in_offs) for f in self.flat_in]
+        self.dev_out = [self._views(f, self.out_shapes, self.out_offs) for f in self.flat_out]
+        self.params = []
+        for din, dout in zip(self.dev_in, self.dev_out):
+            extra = {"positions": din["positions"]} if "positions" in din else {}
+            if "q_scale" in dout:
+                extra["q_scale"] = dout["q_scale"]
+            self.params.append(append_params(din["qkv"], cos_sin_cache, din["q_indptr"],
+                                             din["seq_lens"], din["page_table"], k_cache, v_cache,
+                                             dout["out_q"], dout["flags"], **extra, **kw))
+        self.s_in = torch.cuda.Stream(device)
+        self.s_k = torch.cuda.Stream(device)
+        self.s_out = torch.cuda.Stream(device)
+        mk = lambda: [torch.cuda.Event() for _ in range(depth)]
+        self.ev_in, self.ev_k, self.ev_out = mk(), mk(), mk()
+        self.used = [False] * depth
+        self.i = 0
+
+    @classmethod
+    def _layout(cls, shapes):
+        import torch
+        offs, n = {}, 0
+        for k, (sh, dt) in shapes.items():
+            offs[k] = n
+            size = int(np.prod(sh)) * torch.empty((), dtype=dt).element_size()
+            n += -(-size // cls._ALIGN) * cls._ALIGN
+        return max(n, cls._ALIGN), offs
+
+    @staticmethod
+    def _views(flat, shapes, offs):
+        import torch
+        out = {}
+        for k, (sh, dt) in shapes.items():
+            size = int(np.prod(sh)) * torch.empty((), dtype=dt).element_size()
+            out[k] = flat[offs[k]:offs[k] + size].view(dt).view(sh)
+        return out
+
+    def new_host_buffers(self):
+        """(host_in, host_out): pinned host views, each set backed by one flat
+        buffer (kept under the key "_flat"), for one-copy submits."""
+        torch = self.torch
+        fin = torch.empty(self.in_bytes, dtype=torch.uint8).pin_memory()
+        fout = torch.empty(self.out_bytes, dtype=torch.uint8).pin_memory()
+        hin = self._views(fin, self.in_shapes, self.in_offs)
+        hout = self._views(fout, self.out_shapes, self.out_offs)
+        hin["_flat"], hout["_flat"] = fin, fout
+        return hin, hout
+
+    def submit(self, host_in: dict, host_out: dict):
+        torch = self.torch
+        j = self.i % self.depth
+        self.i += 1
+        with torch.cuda.stream(self.s_in):
+            if self.used[j]:
+                self.s_in.wait_event(self.ev_k[j])        # slot j's inputs consumed
+            if "_flat" in host_in:
+                self.flat_in[j].copy_(host_in["_flat"], non_blocking=True)
+            else:
+                for k, h in host_in.items():
+                    self.dev_in[j][k].copy_(h, non_blocking=True)
+            self.ev_in[j].record(self.s_in)
+        self.s_k.wait_event(self.ev_in[j])
+        if self.used[j]:
+            self.s_k.wait_event(self.ev_out[j])           # slot j's results copied out
+        rc = append_paged_raw(self.params[j], self.s_k.cuda_stream)
+        if rc != FQR_OK:
+            raise FqrError(rc)
+        self.ev_k[j].record(self.s_k)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(self.ev_k[j])
+            if "_flat" in host_out:
+                host_out["_flat"].copy_(self.flat_out[j], non_blocking=True)
+            else:
+                for k, h in host_out.items():
+                    h.copy_(self.dev_out[j][k], non_blocking=True)
+            self.ev_out[j].record(self.s_out)
+        self.used[j] = True
+        return self.ev_out[j]
+
+    def synchronize(self):
+        for s in (self.s_in, self.s_k, self.s_out):
+            s.synchronize()
+
+
 def mla_params(q, kv_c, k_pe, cos_sin_cache, q_indptr, seq_lens, block_table, latent_cache,
                flags, *, nope_dim: int, rope_style: int = 1, kv_scale=None,
                positions=None, q_quant: int = MLA_Q_NONE, q_scale_inv=None,
@@ -228,7 +348,7 @@ def concat_mla_cache(q, kv_c, k_pe, cos_sin_cache, q_indptr, seq_lens, block_tab
 
 
 __all__ = ["LIB", "LIB_PATH", "AppendParams", "MlaParams", "FqrError", "strerror",
-           "append_paged_from_host",
+           "append_paged_from_host", "StagedAppend",
            "append_params", "append_paged", "append_paged_raw", "mla_params",
            "concat_mla_cache", "concat_mla_cache_raw", "FQR_OK", "FQR_EINVAL",
            "FQR_ENOTSUP", "FQR_ECUDA", "HEAD_DIM", "MAX_BATCH", "SCHEDULE_AUTO",
