@@ -407,31 +407,27 @@ def e2e_measure(torch, fqr, bench, steps):
     h2d = int(host_in[0]["_flat"].numel())
     d2h = int(host_out[0]["_flat"].numel())
 
-    def step(i):
-        return sa.submit(host_in[i % R], host_out[i % R])
-
     for i in range(20):
-        step(i)
+        sa.submit(host_in[i % R], host_out[i % R])
     sa.synchronize()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for st in (sa.s_in, sa.s_k, sa.s_out):
-        st.wait_event(start)
-    last = None
+    sa.fork(stream)           # the pipeline's streams start after `start`
     for i in range(steps):
-        last = step(i)
-    stream.wait_event(last)   # the last copy-out follows every earlier step's work
+        sa.submit(host_in[i % R], host_out[i % R])
+    sa.join(stream)           # `end` follows every step's copy-out
     end.record(stream)
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
     assert int(host_out[(steps - 1) % R]["flags"].abs().max()) == 0
+    sa.close()
     return {"value": bench.T * steps / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps,
-            "api": "qk_norm_rope_token_b200.StagedAppend (3 streams, 3 staging buffers, one "
-                   "flat pinned buffer each way)"}
+            "api": "qk_norm_rope_token_b200.StagedAppend over the library's native pipeline "
+                   "(fqr_pipeline_*: 3 streams, 3 staging slots, one copy each way per step)"}
 
 
 # ----------------------------------------------------------- CPU baselines

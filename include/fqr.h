@@ -28,6 +28,7 @@
 #ifndef FQR_H
 #define FQR_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -175,6 +176,46 @@ typedef struct fqr_append_params {
 } fqr_append_params;
 
 int fqr_append_paged(const fqr_append_params* p, void* stream);
+
+/*
+ * fqr_pipeline_* -- fqr_append_paged on batches held in pinned host memory,
+ * pipelined.  A pipeline has `depth` slots; slot j owns a device input buffer
+ * dev_in[j] (in_bytes) and a device result buffer dev_out[j] (out_bytes),
+ * allocated by the caller, and a parameter block params[j] whose device
+ * pointers point into them (qkv and metadata into dev_in[j]; out_q, flags,
+ * q_scale into dev_out[j]) or at resident device data (caches, cos/sin,
+ * weights, scales).  Each submit, for the next slot in turn, enqueues on
+ * three streams the pipeline owns:
+ *   copy-in:  host_in (in_bytes, pinned) -> dev_in[j], once slot j's
+ *             previous kernel has run;
+ *   compute:  fqr_append_paged(params[j]), after that copy and once slot j's
+ *             previous results have been copied out;
+ *   copy-out: dev_out[j] -> host_out (out_bytes, pinned).
+ * So the copy-in of one batch, the kernel of the one before and the copy-out
+ * of the one before that overlap.  One host->device and one device->host copy
+ * per batch (cudaMemcpyAsync each); no device memory is allocated.
+ *
+ * create: checks every params[j] as fqr_append_paged does (T = B = 0 is
+ *   rejected), creates three non-blocking streams and 3*depth events on the
+ *   current device; *out receives the handle.  FQR_EINVAL / FQR_ENOTSUP /
+ *   FQR_ECUDA, with *out = NULL, on failure.
+ * submit: asynchronous; host buffers must stay valid until the batch is
+ *   done (fqr_pipeline_sync, or a stream that fqr_pipeline_join made wait).
+ * fork: the pipeline's streams wait for the work enqueued so far on `stream`.
+ * join: `stream` waits for every batch submitted so far.
+ * sync: blocks the host until every submitted batch is done.
+ * destroy: syncs, then releases the streams and events.
+ */
+#define FQR_PIPELINE_MAX_DEPTH 8
+typedef struct fqr_pipeline fqr_pipeline;
+int fqr_pipeline_create(int depth, const fqr_append_params* params, void* const* dev_in,
+                        size_t in_bytes, void* const* dev_out, size_t out_bytes,
+                        fqr_pipeline** out);
+int fqr_pipeline_submit(fqr_pipeline* p, const void* host_in, void* host_out);
+int fqr_pipeline_fork(fqr_pipeline* p, void* stream);
+int fqr_pipeline_join(fqr_pipeline* p, void* stream);
+int fqr_pipeline_sync(fqr_pipeline* p);
+int fqr_pipeline_destroy(fqr_pipeline* p);
 
 /*
  * fqr_concat_mla_cache -- MLA variant: rotate the rope part of Q in place and

@@ -80,6 +80,18 @@ def _load() -> ctypes.CDLL:
     lib.fqr_concat_mla_cache.restype = ctypes.c_int
     lib.fqr_strerror.argtypes = [ctypes.c_int]
     lib.fqr_strerror.restype = ctypes.c_char_p
+    lib.fqr_pipeline_create.argtypes = [ctypes.c_int, ctypes.POINTER(AppendParams),
+                                        ctypes.POINTER(c_vp), ctypes.c_size_t,
+                                        ctypes.POINTER(c_vp), ctypes.c_size_t,
+                                        ctypes.POINTER(c_vp)]
+    for name in ("fqr_pipeline_create", "fqr_pipeline_submit", "fqr_pipeline_fork",
+                 "fqr_pipeline_join", "fqr_pipeline_sync", "fqr_pipeline_destroy"):
+        getattr(lib, name).restype = ctypes.c_int
+    lib.fqr_pipeline_submit.argtypes = [c_vp, c_vp, c_vp]
+    lib.fqr_pipeline_fork.argtypes = [c_vp, c_vp]
+    lib.fqr_pipeline_join.argtypes = [c_vp, c_vp]
+    lib.fqr_pipeline_sync.argtypes = [c_vp]
+    lib.fqr_pipeline_destroy.argtypes = [c_vp]
     return lib
 
 
@@ -195,25 +207,25 @@ def append_paged_from_host(host_in: dict, dev_in: dict, host_out: dict, dev_out:
 
 
 class StagedAppend:
-    """append_paged on batches that live in pinned host memory, pipelined.
+    """append_paged on batches that live in pinned host memory, pipelined by
+    the library's native pipeline (fqr_pipeline_* in include/fqr.h).
 
     Each submit() enqueues, for one batch: the host-to-device copy of its
-    inputs on a copy-in stream, the fused kernel on a compute stream, and the
-    device-to-host copy of its results on a copy-out stream, with events
-    between them and `depth` sets of device staging buffers rotated.  So the
-    copy-in of the next batch, the kernel of this one and the copy-out of the
-    previous one overlap (PCIe carries both directions at once).
+    inputs, the fused kernel and the device-to-host copy of its results, on
+    three streams with events between them and `depth` sets of device staging
+    buffers rotated.  So the copy-in of the next batch, the kernel of this one
+    and the copy-out of the previous one overlap (PCIe carries both directions
+    at once).
 
     in_shapes / out_shapes map the names of append_paged_from_host ("qkv",
     "q_indptr", "seq_lens", "page_table", optionally "positions"; "out_q",
-    "flags", optionally "q_scale") to (shape, dtype).  Each slot's inputs
-    (and results) are views of one flat device buffer, so host buffers made
-    by new_host_buffers() -- views of one flat pinned buffer -- move in one
-    copy each way.  The KV caches, cos/sin cache, norm weights and the other
-    append_paged keywords are fixed at construction (each slot's parameter
-    block is built once).  synchronize() waits for every submitted batch;
-    read a batch's host results after that, or after the event submit()
-    returns."""
+    "flags", optionally "q_scale") to (shape, dtype).  Each slot's inputs (and
+    results) are views of one flat device buffer; new_host_buffers() returns
+    matching pinned host views of one flat buffer each way, so a batch moves
+    in one copy each way.  The KV caches, cos/sin cache, norm weights and the
+    other append_paged keywords are fixed at construction.  synchronize()
+    waits for every submitted batch; join(stream) makes a stream wait for
+    them."""
 
     _ALIGN = 256
 
@@ -230,21 +242,24 @@ class StagedAppend:
                          for _ in range(depth)]
         self.dev_in = [self._views(f, self.in_shapes, self.in_offs) for f in self.flat_in]
         self.dev_out = [self._views(f, self.out_shapes, self.out_offs) for f in self.flat_out]
-        self.params = []
+        params = []
         for din, dout in zip(self.dev_in, self.dev_out):
             extra = {"positions": din["positions"]} if "positions" in din else {}
             if "q_scale" in dout:
                 extra["q_scale"] = dout["q_scale"]
-            self.params.append(append_params(din["qkv"], cos_sin_cache, din["q_indptr"],
-                                             din["seq_lens"], din["page_table"], k_cache, v_cache,
-                                             dout["out_q"], dout["flags"], **extra, **kw))
-        self.s_in = torch.cuda.Stream(device)
-        self.s_k = torch.cuda.Stream(device)
-        self.s_out = torch.cuda.Stream(device)
-        mk = lambda: [torch.cuda.Event() for _ in range(depth)]
-        self.ev_in, self.ev_k, self.ev_out = mk(), mk(), mk()
-        self.used = [False] * depth
-        self.i = 0
+            params.append(append_params(din["qkv"], cos_sin_cache, din["q_indptr"],
+                                        din["seq_lens"], din["page_table"], k_cache, v_cache,
+                                        dout["out_q"], dout["flags"], **extra, **kw))
+        self._keep = (cos_sin_cache, k_cache, v_cache, kw)
+        self._params = (AppendParams * depth)(*params)
+        dev_in = (c_vp * depth)(*[f.data_ptr() for f in self.flat_in])
+        dev_out = (c_vp * depth)(*[f.data_ptr() for f in self.flat_out])
+        self._handle = c_vp()
+        rc = LIB.fqr_pipeline_create(depth, self._params, dev_in, self.in_bytes, dev_out,
+                                     self.out_bytes, ctypes.byref(self._handle))
+        if rc != FQR_OK:
+            self._handle = None
+            raise FqrError(rc)
 
     @classmethod
     def _layout(cls, shapes):
@@ -267,7 +282,7 @@ class StagedAppend:
 
     def new_host_buffers(self):
         """(host_in, host_out): pinned host views, each set backed by one flat
-        buffer (kept under the key "_flat"), for one-copy submits."""
+        buffer (kept under the key "_flat")."""
         torch = self.torch
         fin = torch.empty(self.in_bytes, dtype=torch.uint8).pin_memory()
         fout = torch.empty(self.out_bytes, dtype=torch.uint8).pin_memory()
@@ -276,40 +291,40 @@ class StagedAppend:
         hin["_flat"], hout["_flat"] = fin, fout
         return hin, hout
 
-    def submit(self, host_in: dict, host_out: dict):
-        torch = self.torch
-        j = self.i % self.depth
-        self.i += 1
-        with torch.cuda.stream(self.s_in):
-            if self.used[j]:
-                self.s_in.wait_event(self.ev_k[j])        # slot j's inputs consumed
-            if "_flat" in host_in:
-                self.flat_in[j].copy_(host_in["_flat"], non_blocking=True)
-            else:
-                for k, h in host_in.items():
-                    self.dev_in[j][k].copy_(h, non_blocking=True)
-            self.ev_in[j].record(self.s_in)
-        self.s_k.wait_event(self.ev_in[j])
-        if self.used[j]:
-            self.s_k.wait_event(self.ev_out[j])           # slot j's results copied out
-        rc = append_paged_raw(self.params[j], self.s_k.cuda_stream)
+    def submit(self, host_in: dict, host_out: dict) -> None:
+        """Enqueue one batch (buffers from new_host_buffers)."""
+        rc = LIB.fqr_pipeline_submit(self._handle, c_vp(host_in["_flat"].data_ptr()),
+                                     c_vp(host_out["_flat"].data_ptr()))
         if rc != FQR_OK:
             raise FqrError(rc)
-        self.ev_k[j].record(self.s_k)
-        with torch.cuda.stream(self.s_out):
-            self.s_out.wait_event(self.ev_k[j])
-            if "_flat" in host_out:
-                host_out["_flat"].copy_(self.flat_out[j], non_blocking=True)
-            else:
-                for k, h in host_out.items():
-                    h.copy_(self.dev_out[j][k], non_blocking=True)
-            self.ev_out[j].record(self.s_out)
-        self.used[j] = True
-        return self.ev_out[j]
 
-    def synchronize(self):
-        for s in (self.s_in, self.s_k, self.s_out):
-            s.synchronize()
+    def fork(self, stream) -> None:
+        """The pipeline's streams wait for the work enqueued so far on `stream`."""
+        rc = LIB.fqr_pipeline_fork(self._handle, c_vp(_stream(stream, None)))
+        if rc != FQR_OK:
+            raise FqrError(rc)
+
+    def join(self, stream) -> None:
+        """`stream` waits for every batch submitted so far."""
+        rc = LIB.fqr_pipeline_join(self._handle, c_vp(_stream(stream, None)))
+        if rc != FQR_OK:
+            raise FqrError(rc)
+
+    def synchronize(self) -> None:
+        rc = LIB.fqr_pipeline_sync(self._handle)
+        if rc != FQR_OK:
+            raise FqrError(rc)
+
+    def close(self) -> None:
+        if self._handle:
+            LIB.fqr_pipeline_destroy(self._handle)
+            self._handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def mla_params(q, kv_c, k_pe, cos_sin_cache, q_indptr, seq_lens, block_table, latent_cache,

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfqr.so")
 SOURCES = ["fqr_api.cu", "fqr_append.cu", "fqr_append_warp.cu", "fqr_append_pipe.cu",
-           "fqr_mla.cu"]
+           "fqr_mla.cu", "fqr_runtime.cu"]
 DEPS = ["fqr_device.cuh", "fqr_head.cuh", "fqr_launch.h"]
 
 NVCC_FLAGS = [

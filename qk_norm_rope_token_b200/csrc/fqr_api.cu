@@ -15,6 +15,10 @@ inline bool aligned(const void* p, uintptr_t n) {
   return (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0;
 }
 
+}  // namespace
+
+namespace fqr {
+
 int check_append(const fqr_append_params* p) {
   if (p == nullptr) return FQR_EINVAL;
   if (p->T < 0 || p->B < 0 || p->B > FQR_MAX_BATCH) return FQR_EINVAL;
@@ -76,6 +80,10 @@ int check_append(const fqr_append_params* p) {
   return FQR_OK;
 }
 
+}  // namespace fqr
+
+namespace {
+
 int check_mla(const fqr_mla_params* p) {
   if (p == nullptr) return FQR_EINVAL;
   if (p->T < 0 || p->B < 0 || p->B > FQR_MAX_BATCH) return FQR_EINVAL;
@@ -129,7 +137,7 @@ extern "C" {
 
 int fqr_append_paged(const fqr_append_params* p, void* stream) {
   if (p != nullptr && p->T == 0 && p->B == 0) return FQR_OK;  // empty batch: no launch
-  const int rc = check_append(p);
+  const int rc = fqr::check_append(p);
   if (rc != FQR_OK) return rc;
   return fqr::launch_append(*p, static_cast<cudaStream_t>(stream));
 }

@@ -391,14 +391,9 @@ int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStr
   a.max_seqlen = p.quant_policy == 1 ? p.max_seqlen : 0;
   a.flags = p.flags;
 
-  int dev = 0, sms = 0, smem_optin = 0, smem_sm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-          cudaSuccess ||
-      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
-          cudaSuccess)
-    return FQR_ECUDA;
+  DeviceInfo d;
+  if (device_info(&d) != FQR_OK) return FQR_ECUDA;
+  const int sms = d.sms, smem_optin = d.smem_optin, smem_sm = d.smem_sm;
 
   const int64_t meta = static_cast<int64_t>(2 * p.B + 1) * sizeof(int);
   auto stage_bytes = [&](int hc) { return kHeader + a.cs_bytes + hc * kHeadDim * 2; };
@@ -426,15 +421,8 @@ int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStr
   const size_t smem = static_cast<size_t>(kFixedSmem + meta + static_cast<int64_t>(S) * a.stage_bytes);
 
   PipeKernel k = select_pipe(p.quant_policy, p.rope_style);
-  const void* fn = reinterpret_cast<const void*>(k);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return FQR_ECUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kPipeThreads, smem) !=
-          cudaSuccess ||
-      per_sm < 1)
+  if (resident_blocks(reinterpret_cast<const void*>(k), kPipeThreads, smem, &per_sm) != FQR_OK)
     return FQR_ECUDA;
   const int64_t cap = static_cast<int64_t>(per_sm) * sms;
   const int64_t want = a.units > sms ? a.units : sms;

@@ -266,19 +266,12 @@ int64_t latency_tasks(const fqr_append_params& p) {
 }
 
 int64_t latency_capacity(const fqr_append_params& p) {
-  int dev = 0, sms = 0, per_sm = 0;
+  DeviceInfo d;
+  int per_sm = 0;
   const void* fn = reinterpret_cast<const void*>(select_warp(p.quant_policy, p.rope_style));
-  const size_t smem = warp_smem(p);
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+  if (device_info(&d) != FQR_OK || resident_blocks(fn, kThreads, warp_smem(p), &per_sm) != FQR_OK)
     return -1;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return -1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem) != cudaSuccess)
-    return -1;
-  return static_cast<int64_t>(per_sm) * sms * kWarps;
+  return static_cast<int64_t>(per_sm) * d.sms * kWarps;
 }
 
 int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream) {

@@ -11,6 +11,8 @@
 namespace fqr {
 
 struct HeadParams;
+// Host-side argument checks of fqr_append_paged (FQR_OK or the error code).
+int check_append(const fqr_append_params* p);
 int launch_append(const fqr_append_params& p, cudaStream_t stream);
 int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream);
 // Warp tasks of the latency schedule for p, and how many warps of it the
@@ -19,6 +21,17 @@ int64_t latency_tasks(const fqr_append_params& p);
 int64_t latency_capacity(const fqr_append_params& p);
 int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream);
 int launch_mla(const fqr_mla_params& p, cudaStream_t stream);
+
+// Launch facts of the current device, cached after the first query
+// (fqr_runtime.cu).
+struct DeviceInfo {
+  int dev, sms, smem_optin, smem_sm;
+};
+int device_info(DeviceInfo* out);
+// Resident blocks per SM of kernel fn at this block size and dynamic shared
+// memory (raising the kernel's dynamic shared-memory limit when smem > 48 KiB),
+// cached per (kernel, threads, smem, device).
+int resident_blocks(const void* fn, int threads, size_t smem, int* per_sm);
 
 // Launch `kernel(args)` on `stream` with programmatic stream serialization,
 // so that it may begin while the preceding kernel in the stream finishes; the
@@ -49,21 +62,13 @@ int launch_pdl(void (*kernel)(const Args), int grid, int threads, size_t smem,
 template <class F>
 int launch_persistent(const void* func, int64_t warp_tasks, size_t smem,
                       cudaStream_t /*stream*/, F&& launch) {
-  int dev = 0, sms = 0, per_sm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FQR_ECUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return FQR_ECUDA;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return FQR_ECUDA;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, func, kThreads, smem) !=
-          cudaSuccess ||
-      per_sm < 1)
+  DeviceInfo d;
+  int per_sm = 0;
+  if (device_info(&d) != FQR_OK || resident_blocks(func, kThreads, smem, &per_sm) != FQR_OK)
     return FQR_ECUDA;
   int64_t need = (warp_tasks + kWarps - 1) / kWarps;
   if (need < 1) need = 1;
-  const int64_t cap = static_cast<int64_t>(per_sm) * sms;
+  const int64_t cap = static_cast<int64_t>(per_sm) * d.sms;
   return launch(static_cast<int>(need < cap ? need : cap));
 }
 

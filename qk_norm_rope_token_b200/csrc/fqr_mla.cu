@@ -552,18 +552,12 @@ int launch_mla(const fqr_mla_params& p, cudaStream_t stream) {
                               : (p.rope_style == 0 ? mla_token_kernel<0, 0> : mla_token_kernel<0, 1>);
     const int nw = a.qgroups < kTokenWarps ? a.qgroups : kTokenWarps;  // warps per block
     const size_t smem = static_cast<size_t>(2 * p.B + 1) * sizeof(int) + nw * sizeof(float);
-    int dev = 0, sms = 0, per_sm = 0;
-    const void* fn = reinterpret_cast<const void*>(k);
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    DeviceInfo d;
+    int per_sm = 0;
+    if (device_info(&d) != FQR_OK ||
+        resident_blocks(reinterpret_cast<const void*>(k), 32 * nw, smem, &per_sm) != FQR_OK)
       return FQR_ECUDA;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return FQR_ECUDA;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, 32 * nw, smem) != cudaSuccess ||
-        per_sm < 1)
-      return FQR_ECUDA;
+    const int sms = d.sms;
     const int64_t cap = static_cast<int64_t>(per_sm) * sms;
     const int64_t want = p.T > 0 ? p.T : 1;
     return launch_pdl(k, static_cast<int>(want < cap ? want : cap), 32 * nw, smem, stream, a);

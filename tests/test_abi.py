@@ -28,7 +28,10 @@ def declared_functions():
 
 
 def test_header_declares_the_entry_points():
-    assert declared_functions() == ["fqr_append_paged", "fqr_concat_mla_cache", "fqr_strerror"]
+    assert declared_functions() == ["fqr_append_paged", "fqr_concat_mla_cache",
+                                    "fqr_pipeline_create", "fqr_pipeline_destroy",
+                                    "fqr_pipeline_fork", "fqr_pipeline_join",
+                                    "fqr_pipeline_submit", "fqr_pipeline_sync", "fqr_strerror"]
 
 
 def test_library_exports_every_declared_symbol(fqr):
@@ -209,3 +212,27 @@ MLA_BAD = {
 def test_mla_host_checks_reject(fqr, case):
     over, code = MLA_BAD[case]
     assert fqr.concat_mla_cache_raw(valid_mla(fqr, **over)) == code
+
+
+def test_pipeline_rejects_bad_arguments_before_any_cuda_call(fqr):
+    import ctypes
+    h = ctypes.c_void_p()
+    good = (fqr.AppendParams * 1)(valid_append(fqr))
+    ptrs = (ctypes.c_void_p * 1)(FAKE)
+    L = fqr.LIB
+    assert L.fqr_pipeline_create(0, good, ptrs, 256, ptrs, 256, ctypes.byref(h)) == fqr.FQR_EINVAL
+    assert L.fqr_pipeline_create(9, good, ptrs, 256, ptrs, 256, ctypes.byref(h)) == fqr.FQR_EINVAL
+    assert L.fqr_pipeline_create(1, None, ptrs, 256, ptrs, 256, ctypes.byref(h)) == fqr.FQR_EINVAL
+    assert L.fqr_pipeline_create(1, good, ptrs, 0, ptrs, 256, ctypes.byref(h)) == fqr.FQR_EINVAL
+    nul = (ctypes.c_void_p * 1)(None)
+    assert L.fqr_pipeline_create(1, good, nul, 256, ptrs, 256, ctypes.byref(h)) == fqr.FQR_EINVAL
+    bad = (fqr.AppendParams * 1)(valid_append(fqr, head_dim=64))
+    assert L.fqr_pipeline_create(1, bad, ptrs, 256, ptrs, 256, ctypes.byref(h)) == fqr.FQR_EINVAL
+    empty = (fqr.AppendParams * 1)(valid_append(fqr, T=0, B=0))
+    assert L.fqr_pipeline_create(1, empty, ptrs, 256, ptrs, 256, ctypes.byref(h)) == fqr.FQR_EINVAL
+    assert not h.value
+    for name in ("fqr_pipeline_sync", "fqr_pipeline_destroy"):
+        assert getattr(L, name)(None) == fqr.FQR_EINVAL
+    assert L.fqr_pipeline_submit(None, FAKE, FAKE) == fqr.FQR_EINVAL
+    assert L.fqr_pipeline_join(None, None) == fqr.FQR_EINVAL
+    assert L.fqr_pipeline_fork(None, None) == fqr.FQR_EINVAL

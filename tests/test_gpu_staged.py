@@ -1,6 +1,7 @@
-"""GPU test of the pipelined host-memory API (StagedAppend): the same batches
-submitted through it give bitwise the same host results and the same caches
-as sequential append_paged calls, for every pipeline depth."""
+"""GPU test of the pipelined host-memory API (StagedAppend over the native
+fqr_pipeline_*): the same batches submitted through it give bitwise the same
+host results and the same caches as sequential append_paged calls, for every
+pipeline depth, and a stream joined after the submits sees them done."""
 import numpy as np
 import pytest
 import torch
@@ -59,7 +60,7 @@ def test_staged_matches_sequential(depth, policy):
         fqr.append_paged(_dev(w.qkv), cs, _dev(w.q_indptr), _dev(w.seq_lens), _dev(w.page_table),
                          *caches["seq"], out_q, flags, q_scale=q_scale, **kw)
         seq_out.append((out_q.cpu(), flags.cpu(), None if q_scale is None else q_scale.cpu()))
-    # pipelined, through flat host buffers and through separate host tensors
+    # pipelined
     in_shapes = {"qkv": ((w0.T, w0.row_stride), torch.int16), "q_indptr": ((w0.B + 1,), torch.int32),
                  "seq_lens": ((w0.B,), torch.int32),
                  "page_table": (tuple(w0.page_table.shape), torch.int32)}
@@ -69,25 +70,51 @@ def test_staged_matches_sequential(depth, policy):
     sa = fqr.StagedAppend(in_shapes, out_shapes, DEV, depth=depth, cos_sin_cache=cs,
                           k_cache=caches["staged"][0], v_cache=caches["staged"][1], **kw)
     host_out = []
-    for i, w in enumerate(ws):
-        if i % 2 == 0:
-            hi, ho = sa.new_host_buffers()
-            hi["qkv"].copy_(torch.from_numpy(w.qkv.view(np.int16)))
-            hi["q_indptr"].copy_(torch.from_numpy(w.q_indptr))
-            hi["seq_lens"].copy_(torch.from_numpy(w.seq_lens))
-            hi["page_table"].copy_(torch.from_numpy(w.page_table))
-        else:
-            hi = {"qkv": torch.from_numpy(w.qkv.view(np.int16)).pin_memory(),
-                  "q_indptr": torch.from_numpy(w.q_indptr).pin_memory(),
-                  "seq_lens": torch.from_numpy(w.seq_lens).pin_memory(),
-                  "page_table": torch.from_numpy(w.page_table).pin_memory()}
-            ho = {k: torch.empty(sh, dtype=dt).pin_memory() for k, (sh, dt) in out_shapes.items()}
+    for w in ws:
+        hi, ho = sa.new_host_buffers()
+        hi["qkv"].copy_(torch.from_numpy(w.qkv.view(np.int16)))
+        hi["q_indptr"].copy_(torch.from_numpy(w.q_indptr))
+        hi["seq_lens"].copy_(torch.from_numpy(w.seq_lens))
+        hi["page_table"].copy_(torch.from_numpy(w.page_table))
         sa.submit(hi, ho)
         host_out.append(ho)
     sa.synchronize()
+    sa.close()
     for (oq, fl, qs), ho in zip(seq_out, host_out):
         assert torch.equal(oq, ho["out_q"]) and torch.equal(fl, ho["flags"])
         if qs is not None:
             assert torch.equal(qs, ho["q_scale"])
     assert torch.equal(caches["seq"][0], caches["staged"][0])
     assert torch.equal(caches["seq"][1], caches["staged"][1])
+
+
+def test_join_orders_a_stream_after_the_batches():
+    ws = _batches(4, 0)
+    w0 = ws[0]
+    shape = (w0.num_pages, w0.page_size, w0.Hkv, 128)
+    kc = torch.zeros(shape, dtype=torch.int16, device=DEV)
+    vc = torch.zeros(shape, dtype=torch.int16, device=DEV)
+    in_shapes = {"qkv": ((w0.T, w0.row_stride), torch.int16), "q_indptr": ((w0.B + 1,), torch.int32),
+                 "seq_lens": ((w0.B,), torch.int32),
+                 "page_table": (tuple(w0.page_table.shape), torch.int32)}
+    out_shapes = {"out_q": ((w0.T, w0.Hq, 128), torch.int16), "flags": ((w0.B,), torch.int32)}
+    sa = fqr.StagedAppend(in_shapes, out_shapes, DEV, depth=2, cos_sin_cache=_dev(w0.cos_sin),
+                          k_cache=kc, v_cache=vc, q_norm_w=_dev(w0.q_norm_w),
+                          k_norm_w=_dev(w0.k_norm_w))
+    hos = []
+    for w in ws:
+        hi, ho = sa.new_host_buffers()
+        hi["qkv"].copy_(torch.from_numpy(w.qkv.view(np.int16)))
+        hi["q_indptr"].copy_(torch.from_numpy(w.q_indptr))
+        hi["seq_lens"].copy_(torch.from_numpy(w.seq_lens))
+        hi["page_table"].copy_(torch.from_numpy(w.page_table))
+        ho["flags"].fill_(77)
+        sa.submit(hi, ho)
+        hos.append(ho)
+    s = torch.cuda.Stream()
+    sa.join(s)
+    ev = torch.cuda.Event()
+    ev.record(s)
+    ev.synchronize()
+    assert all(int(ho["flags"].abs().max()) == 0 for ho in hos)
+    sa.close()
