@@ -2,8 +2,8 @@
 
 Every step of the path runs in the library's CUDA kernels; PyTorch supplies
 device memory and the stream.  There is no fallback: importing this package
-fails if the library has not been built (python -m
-qk_norm_rope_token_b200.build).
+fails if the library has not been built (python
+qk_norm_rope_token_b200/build.py).
 
     append_paged(...)       -> fqr_append_paged
     concat_mla_cache(...)   -> fqr_concat_mla_cache
@@ -71,7 +71,7 @@ class MlaParams(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m qk_norm_rope_token_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python qk_norm_rope_token_b200/build.py` "
             "(there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     lib.fqr_append_paged.argtypes = [ctypes.POINTER(AppendParams), c_vp]

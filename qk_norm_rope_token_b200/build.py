@@ -1,6 +1,6 @@
 """Build libfqr.so (the CUDA library behind include/fqr.h) for sm_100a.
 
-    python -m qk_norm_rope_token_b200.build [--force] [--verbose-ptxas]
+    python qk_norm_rope_token_b200/build.py [--force] [--verbose-ptxas]
 
 nvcc cross-compiles on a machine without a GPU.  The library is built in-tree
 (qk_norm_rope_token_b200/libfqr.so) with the CUDA runtime linked statically.

@@ -15,7 +15,11 @@ HEADER = os.path.join(ROOT, "include", "fqr.h")
 
 @pytest.fixture(scope="module")
 def fqr():
-    from qk_norm_rope_token_b200 import build
+    import importlib.util
+    path = os.path.join(ROOT, "qk_norm_rope_token_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_fqr_lib_build", path)
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)  # by path: the package refuses to import before the build
     build.build()
     import qk_norm_rope_token_b200 as m
     return m
