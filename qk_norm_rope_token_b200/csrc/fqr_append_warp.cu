@@ -62,8 +62,9 @@ __device__ __forceinline__ void warp_load_head(const WarpArgs& a, int w, int g, 
   }
 }
 
-template <int POLICY, int STYLE>
-__global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a) {
+template <int POLICY, int STYLE, int NT>
+__global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
+  constexpr int NW = NT / 32;  // warps per block
   extern __shared__ __align__(16) int smem[];
   float* s_w = reinterpret_cast<float*>(smem);  // 256 fp32 weights
   int* s_indptr = smem + 2 * kHeadDim;          // B + 1
@@ -77,8 +78,8 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
   const int g = lane >> 3, l8 = lane & 7;
   const unsigned gmask = 0xFFu << (8 * g);
-  const int gwarp = blockIdx.x * kWarps + warp;
-  const int nwarps = gridDim.x * kWarps;
+  const int gwarp = blockIdx.x * NW + warp;
+  const int nwarps = gridDim.x * NW;
 
   const bool paged = a.hp.out_k == nullptr;
   // The first task's coordinates need only the kernel parameters: computed
@@ -146,7 +147,7 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
   // heads and its own request's metadata (request guessed as b = t: one new
   // row per request, the decode case).
   const MetaRegs meta = meta_prefetch(a.q_indptr, a.seq_lens, a.B);
-  const float wreg = weight_prefetch(a.qw, a.kw, a.hp.gemma);
+  const WeightRegs<NT> wreg = weight_prefetch_nt<NT>(a.qw, a.kw, a.hp.gemma);
   uint4 pa = make_uint4(0u, 0u, 0u, 0u), pb = pa;
   int e_lo = 0, e_hi = 0, e_L = 0;
   int64_t e_pos = 0;
@@ -183,7 +184,7 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
         load_cs<STYLE, false>(a.cs + pos * a.hp.rot, a.hp.rot, l8, c0, s0);
     }
   }
-  weight_store(s_w, wreg);
+  weight_store_nt<NT>(s_w, wreg);
   if (a.bulk_tail) zero_buffer_init(s_zero);  // (the prologue's barrier follows)
   bool issued = false;                        // bulk copies in flight (lane 0)
 
@@ -246,15 +247,21 @@ __global__ void __launch_bounds__(kThreads) warp_append_kernel(const WarpArgs a)
 
 using WarpKernel = void (*)(const WarpArgs);
 
-static WarpKernel select_warp(int policy, int style) {
+template <int NT>
+static WarpKernel select_warp_nt(int policy, int style) {
   if (style == 0) {
-    if (policy == 0) return warp_append_kernel<0, 0>;
-    if (policy == 1) return warp_append_kernel<1, 0>;
-    return warp_append_kernel<2, 0>;
+    if (policy == 0) return warp_append_kernel<0, 0, NT>;
+    if (policy == 1) return warp_append_kernel<1, 0, NT>;
+    return warp_append_kernel<2, 0, NT>;
   }
-  if (policy == 0) return warp_append_kernel<0, 1>;
-  if (policy == 1) return warp_append_kernel<1, 1>;
-  return warp_append_kernel<2, 1>;
+  if (policy == 0) return warp_append_kernel<0, 1, NT>;
+  if (policy == 1) return warp_append_kernel<1, 1, NT>;
+  return warp_append_kernel<2, 1, NT>;
+}
+
+static WarpKernel select_warp(int policy, int style, int nt) {
+  return nt == kWideThreads ? select_warp_nt<kWideThreads>(policy, style)
+                            : select_warp_nt<kThreads>(policy, style);
 }
 
 static size_t warp_smem(const fqr_append_params& p) {
@@ -265,13 +272,35 @@ int64_t latency_tasks(const fqr_append_params& p) {
   return static_cast<int64_t>(p.T) * ((p.Hq + 2 * p.Hkv + 3) / 4) + p.B;
 }
 
+// Threads per block of the latency schedule.  Blocks of kThreads while one
+// pass of them leaves every SM at most one block; when it would put two
+// blocks on some SMs and one on the others, and one block of kWideThreads
+// per SM holds every task, the wide block spreads the warps evenly: an SM
+// with twice the warps of its neighbours takes longer in every phase of the
+// launch (load round trips, prologue, stores), and it sets the launch time.
+// Measured on B200 (paged BF16 decode, Hq/Hkv 32/8, page 16, 128 requests:
+// 1,664 warp tasks): 4.04 us per launch with 208 blocks of 8 warps (60 SMs
+// with 16 warps), 3.81 us with 139 blocks of 12.  Without request tails
+// (caller-owned K/V) the launch is short enough that the wide block's lost
+// residency overlap costs more than it gains, so those keep kThreads.
+int warp_block_threads(const fqr_append_params& p) {
+  DeviceInfo d;
+  if (device_info(&d) != FQR_OK) return kThreads;
+  const int64_t tasks = latency_tasks(p);
+  const int64_t narrow_blocks = (tasks + kWarps - 1) / kWarps;
+  const int64_t wide_blocks = (tasks + kWideThreads / 32 - 1) / (kWideThreads / 32);
+  const bool paged = p.out_k == nullptr;
+  return paged && narrow_blocks > d.sms && wide_blocks <= d.sms ? kWideThreads : kThreads;
+}
+
 int64_t latency_capacity(const fqr_append_params& p) {
   DeviceInfo d;
   int per_sm = 0;
-  const void* fn = reinterpret_cast<const void*>(select_warp(p.quant_policy, p.rope_style));
-  if (device_info(&d) != FQR_OK || resident_blocks(fn, kThreads, warp_smem(p), &per_sm) != FQR_OK)
+  const int nt = kThreads;  // (the wide block only serves grids of at most one block per SM)
+  const void* fn = reinterpret_cast<const void*>(select_warp(p.quant_policy, p.rope_style, nt));
+  if (device_info(&d) != FQR_OK || resident_blocks(fn, nt, warp_smem(p), &per_sm) != FQR_OK)
     return -1;
-  return static_cast<int64_t>(per_sm) * d.sms * kWarps;
+  return static_cast<int64_t>(per_sm) * d.sms * (nt / 32);
 }
 
 int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream) {
@@ -300,13 +329,16 @@ int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStr
   a.max_seqlen = p.quant_policy == 1 ? p.max_seqlen : 0;
   a.flags = p.flags;
   const size_t smem = warp_smem(p);
-  WarpKernel k = select_warp(p.quant_policy, p.rope_style);
-  return launch_persistent(reinterpret_cast<const void*>(k), n_head + p.B, smem, stream,
-                           [&](int grid) {
-                             // bulk tails once warps have more than one task
-                             a.bulk_tail = static_cast<int64_t>(grid) * kWarps < n_head + p.B;
-                             return launch_pdl(k, grid, kThreads, smem, stream, a);
-                           });
+  const int nt = warp_block_threads(p);
+  WarpKernel k = select_warp(p.quant_policy, p.rope_style, nt);
+  return launch_persistent(
+      reinterpret_cast<const void*>(k), n_head + p.B, smem, stream,
+      [&](int grid) {
+        // bulk tails once warps have more than one task
+        a.bulk_tail = static_cast<int64_t>(grid) * (nt / 32) < n_head + p.B;
+        return launch_pdl(k, grid, nt, smem, stream, a);
+      },
+      nt);
 }
 
 }  // namespace fqr

@@ -88,18 +88,44 @@ __device__ __forceinline__ int weight_slot(int e) {
 // For blocks of at least 256 threads: weight_prefetch loads one value per
 // thread at kernel entry, weight_store writes it after the first round trip.
 // gemma: the Gemma-style norm scales by 1 + w (an fp32 add) instead of w.
-__device__ __forceinline__ float weight_prefetch(const uint16_t* qw, const uint16_t* kw,
-                                                 int gemma) {
-  const int i = threadIdx.x;
+__device__ __forceinline__ float weight_value(const uint16_t* qw, const uint16_t* kw, int gemma,
+                                              int i) {
   if (i >= 2 * kHeadDim) return 0.0f;
   const uint16_t* w = i < kHeadDim ? qw : kw;
   if (w == nullptr) return 1.0f;  // (the norm is off for this tensor)
   const float v = __uint_as_float(static_cast<uint32_t>(__ldg(w + (i & (kHeadDim - 1)))) << 16);
   return gemma ? __fadd_rn(1.0f, v) : v;
 }
-__device__ __forceinline__ void weight_store(float* s_w, float v) {
-  const int i = threadIdx.x;
+__device__ __forceinline__ void weight_store_at(float* s_w, float v, int i) {
   if (i < 2 * kHeadDim) s_w[(i & kHeadDim) + weight_slot(i & (kHeadDim - 1))] = v;
+}
+__device__ __forceinline__ float weight_prefetch(const uint16_t* qw, const uint16_t* kw,
+                                                 int gemma) {
+  return weight_value(qw, kw, gemma, threadIdx.x);
+}
+__device__ __forceinline__ void weight_store(float* s_w, float v) {
+  weight_store_at(s_w, v, threadIdx.x);
+}
+// The same for blocks of NT threads: 256 / NT values per thread when NT < 256.
+template <int NT>
+struct WeightRegs {
+  static constexpr int kN = NT >= 2 * kHeadDim ? 1 : 2 * kHeadDim / NT;
+  float v[kN];
+};
+template <int NT>
+__device__ __forceinline__ WeightRegs<NT> weight_prefetch_nt(const uint16_t* qw,
+                                                             const uint16_t* kw, int gemma) {
+  WeightRegs<NT> r;
+#pragma unroll
+  for (int k = 0; k < WeightRegs<NT>::kN; ++k)
+    r.v[k] = weight_value(qw, kw, gemma, static_cast<int>(threadIdx.x) + k * NT);
+  return r;
+}
+template <int NT>
+__device__ __forceinline__ void weight_store_nt(float* s_w, const WeightRegs<NT>& r) {
+#pragma unroll
+  for (int k = 0; k < WeightRegs<NT>::kN; ++k)
+    weight_store_at(s_w, r.v[k], static_cast<int>(threadIdx.x) + k * NT);
 }
 
 __device__ __forceinline__ void unpack_pairs(uint4 xa, uint4 xb, float2* y) {

@@ -19,6 +19,8 @@ int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStr
 // device holds at once (-1 if the runtime cannot tell).
 int64_t latency_tasks(const fqr_append_params& p);
 int64_t latency_capacity(const fqr_append_params& p);
+// Threads per block the latency schedule uses for p (fqr_append_warp.cu).
+int warp_block_threads(const fqr_append_params& p);
 int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream);
 int launch_mla(const fqr_mla_params& p, cudaStream_t stream);
 
@@ -56,17 +58,19 @@ int launch_pdl(void (*kernel)(const Args), int grid, int threads, size_t smem,
   return cudaGetLastError() == cudaSuccess ? FQR_OK : FQR_ECUDA;
 }
 
-// Launch a persistent warp-task kernel: one block of kThreads per kWarps
-// tasks, capped at the number of blocks that can be resident on the device at
-// once (the kernel loops over the rest).  `launch(grid)` issues the <<<>>>.
+// Launch a persistent warp-task kernel: one block of `threads` per
+// threads / 32 tasks, capped at the number of blocks that can be resident on
+// the device at once (the kernel loops over the rest).  `launch(grid)` issues
+// the <<<>>>.
 template <class F>
 int launch_persistent(const void* func, int64_t warp_tasks, size_t smem,
-                      cudaStream_t /*stream*/, F&& launch) {
+                      cudaStream_t /*stream*/, F&& launch, int threads = kThreads) {
   DeviceInfo d;
   int per_sm = 0;
-  if (device_info(&d) != FQR_OK || resident_blocks(func, kThreads, smem, &per_sm) != FQR_OK)
+  if (device_info(&d) != FQR_OK || resident_blocks(func, threads, smem, &per_sm) != FQR_OK)
     return FQR_ECUDA;
-  int64_t need = (warp_tasks + kWarps - 1) / kWarps;
+  const int warps = threads / 32;
+  int64_t need = (warp_tasks + warps - 1) / warps;
   if (need < 1) need = 1;
   const int64_t cap = static_cast<int64_t>(per_sm) * d.sms;
   return launch(static_cast<int>(need < cap ? need : cap));

@@ -139,6 +139,46 @@ def test_explicit_position_out_of_range_writes_nothing(bad, schedule):
     assert r.check() == {"flagged": True}
 
 
+def _wide_block_decode(policy, style, B=128, seed=21):
+    """A decode batch of 1,664 latency-schedule warp tasks (128 rows of 12
+    quads, plus 128 request tasks): 208 blocks of 8 warps would leave some SMs
+    with two blocks, 139 blocks of 12 fit one per SM, so the latency schedule
+    takes its wide (12-warp) block here."""
+    rng = np.random.default_rng(seed + policy + 3 * style)
+    L = rng.integers(1, 400, B)
+    return workloads.make_append(seed=seed + policy + 3 * style, n_new=[1] * B, seq_lens=L,
+                                 Hq=32, Hkv=8, page_size=16, max_pages=32,
+                                 quant_policy=policy, rope_style=style, cos_sin_rows=400,
+                                 q_scale_inv=20.0, k_scale=0.05, v_scale=0.05,
+                                 qkv_sigma=2.0 if policy else 1.0)
+
+
+def test_wide_block_preconditions_hold_on_this_device():
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    tasks = 128 * 12 + 128
+    assert -(-tasks // 8) > sms and -(-tasks // 12) <= sms, sms
+
+
+@pytest.mark.parametrize("style", [0, 1])
+@pytest.mark.parametrize("policy", [0, 1, 2])
+def test_wide_block_decode_parity(policy, style):
+    run_and_check(_wide_block_decode(policy, style), schedule=1)
+
+
+@pytest.mark.parametrize("case", ["non_monotone", "page_table_overrun"])
+def test_wide_block_malformed_writes_nothing(case):
+    w = _wide_block_decode(1, 0)
+    ind, L = w.q_indptr.copy(), w.seq_lens.copy()
+    if case == "non_monotone":
+        ind[60] = ind[62]
+    else:
+        L[77] = w.page_size * w.max_pages + 1
+    r = AppendRun(w, schedule=1, q_indptr=ind, seq_lens=L)
+    r.launch()
+    assert r.check() == {"flagged": True}
+    assert (r.flags.cpu().numpy() == -1).all()
+
+
 @pytest.mark.parametrize("schedule", SCHEDULES)
 def test_largest_batch(schedule):
     B = 16384
