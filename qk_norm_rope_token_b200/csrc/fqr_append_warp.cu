@@ -62,6 +62,27 @@ __device__ __forceinline__ void warp_load_head(const WarpArgs& a, int w, int g, 
   }
 }
 
+// Pull into L2 the lines task w's second round trip will read -- its
+// page-table entry and its row's cos/sin values -- while the warp still works
+// on its current task (the request comes from the staged q_indptr, so this
+// runs after the prologue).  A warp with several tasks otherwise pays a full
+// DRAM round trip for these at the start of each later task.
+__device__ __forceinline__ void prefetch_task_lines(const WarpArgs& a, int w, const int* s_indptr,
+                                                    const int* s_seq, int lane, bool paged) {
+  const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
+  const int h0 = (w - t * a.quads) * 4;
+  const int b = request_of_row(s_indptr, a.B, t);
+  const int end = s_indptr[b + 1];
+  const int p_slot = t + s_seq[b] - end;
+  if (lane == 0) {
+    if (paged && (h0 + 3 >= a.hp.Hq || t == end - 1))
+      prefetch_l2(a.page_table + static_cast<int64_t>(b) * a.max_pages +
+                  a.hp.pdiv.div(static_cast<uint32_t>(p_slot)));
+  } else if (a.positions == nullptr && 32 * (lane - 1) < a.hp.rot && h0 < a.hp.Hq + a.hp.Hkv) {
+    prefetch_l2(a.cs + static_cast<int64_t>(p_slot) * a.hp.rot + 32 * (lane - 1));
+  }
+}
+
 template <int POLICY, int STYLE, int NT>
 __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
   constexpr int NW = NT / 32;  // warps per block
@@ -196,7 +217,10 @@ __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
   for (int w = gwarp; w < n_tasks; w += nwarps) {
     if (w < a.n_head) {
       const uint4 xa = pa, xb = pb;
-      if (w + nwarps < a.n_head) warp_load_head(a, w + nwarps, g, l8, pa, pb);
+      if (w + nwarps < a.n_head) {
+        warp_load_head(a, w + nwarps, g, l8, pa, pb);
+        prefetch_task_lines(a, w + nwarps, s_indptr, s_seq, lane, paged);
+      }
       const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
       const int quad = w - t * a.quads;
       if (w == gwarp && early) {  // the batch is valid: the early lookups stand
