@@ -18,7 +18,10 @@
 //     tail (both caches) evenly between them and store their share of zeros
 //     before their heads (the stores drain while the heads are computed);
 //     one "request task" per request zeroes the tail of requests that append
-//     nothing.
+//     nothing -- or, when tails are small and every warp holds one task,
+//     every request's whole tail, so that the head tasks share none.
+//   * blocks of 8 warps, or of 12 when that spreads a one-pass grid evenly
+//     over the SMs (warp_block_threads).
 #include "fqr_head.cuh"
 #include "fqr_launch.h"
 
@@ -42,6 +45,7 @@ struct WarpArgs {
   int64_t slot_cap;  // max_pages * page_size; INT64_MAX with caller-owned K/V
   int max_seqlen;    // > 0: the dynamic-Q prefill check n_b <= max_seqlen
   int bulk_tail;     // tails by bulk copies (warps with several tasks)
+  int own_tails;     // request tasks zero whole tails (head tasks share none)
   int32_t* flags;
 };
 
@@ -199,7 +203,7 @@ __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
       r0.is_last = t0 == e_hi - 1;
       r0.qs = q_scale_row(a.hp, t0, gb, t0 - e_lo);
       // K/V slot, or the tail share of the last row
-      if (paged && (h0 >= a.hp.Hq || r0.is_last))
+      if (paged && (h0 >= a.hp.Hq || (r0.is_last && !a.own_tails)))
         r0.page = __ldg(a.page_table + static_cast<int64_t>(gb) * a.max_pages + pidx);
       if (h0 < a.hp.Hq + a.hp.Hkv)
         load_cs<STYLE, false>(a.cs + pos * a.hp.rot, a.hp.rot, l8, c0, s0);
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
       if (w == gwarp && early) {  // the batch is valid: the early lookups stand
         // (the tail stores need nothing from the head: issue them first so they
         // drain while the head is computed)
-        if (paged && r0.is_last) {
+        if (paged && r0.is_last && !a.own_tails) {
           if (a.bulk_tail)
             issued |= zero_tail_share_bulk(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane, s_zero);
           else
@@ -246,10 +250,11 @@ __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
       r.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : p_slot;
       r.is_last = t == end - 1;
       r.qs = q_scale_row(a.hp, t, b, t - s_indptr[b]);
-      r.page = paged && (h >= a.hp.Hq || r.is_last)
+      const bool share = paged && r.is_last && !a.own_tails;
+      r.page = paged && (h >= a.hp.Hq || share)
                    ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx)
                    : 0;
-      if (paged && r.is_last) {
+      if (share) {
         if (a.bulk_tail)
           issued |= zero_tail_share_bulk(a.hp, r.page, r.slot_row, quad, a.qdiv, lane, s_zero);
         else
@@ -260,9 +265,11 @@ __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
       process_quad<POLICY, STYLE, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, s_w, l8,
                                          gmask);
     } else {
-      const int b = w - a.n_head;  // request task: tail of a request without new rows
+      // request task: the tail of a request without new rows (whose tail no
+      // head task shares), or of every request when request tasks own tails
+      const int b = w - a.n_head;
       const int L = s_seq[b];
-      if (paged && s_indptr[b] == s_indptr[b + 1] && L > 0)
+      if (paged && L > 0 && (a.own_tails || s_indptr[b] == s_indptr[b + 1]))
         zero_request_tail<POLICY == 0 ? 2 : 1>(a.hp, a.page_table, a.max_pages, b, L, lane);
     }
   }
@@ -327,6 +334,16 @@ int64_t latency_capacity(const fqr_append_params& p) {
   return static_cast<int64_t>(per_sm) * d.sms * (nt / 32);
 }
 
+// Request tasks zero whole tails (and the head tasks none) when every warp
+// holds one task and a request's expected tail, (P - 1) / 2 rows of both
+// caches, is at most this many bytes: one warp then writes it in a few
+// stores while the heads run without a tail share.  Larger tails are split
+// over the warps of the request's last row.  Measured on B200 (decode, one
+// row per request): Hq/Hkv 8/1, page 16 (3.75 KiB): 2.99 -> 2.47 us at 1
+// request, 3.50 -> 2.86 us at 128; Hq/Hkv 32/8, page 16 (30 KiB): 2.75 ->
+// 3.57 us at 4 requests with whole tails, so those keep the shares.
+constexpr int64_t kOwnTailsMaxBytes = 4096;
+
 int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream) {
   WarpArgs a;
   a.hp = hp;
@@ -360,6 +377,8 @@ int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStr
       [&](int grid) {
         // bulk tails once warps have more than one task
         a.bulk_tail = static_cast<int64_t>(grid) * (nt / 32) < n_head + p.B;
+        a.own_tails = !a.bulk_tail && static_cast<int64_t>(p.page_size - 1) * hp.row_bytes <=
+                                          kOwnTailsMaxBytes;
         return launch_pdl(k, grid, nt, smem, stream, a);
       },
       nt);

@@ -179,6 +179,20 @@ def test_wide_block_malformed_writes_nothing(case):
     assert (r.flags.cpu().numpy() == -1).all()
 
 
+@pytest.mark.parametrize("policy", [0, 1, 2])
+def test_small_tails_owned_by_request_tasks(policy):
+    """Tails of at most 4 KiB per request (Hkv 1, page 16) in a one-pass
+    latency launch: request tasks zero whole tails, including those of
+    requests without new rows and of requests with several rows."""
+    n = [1, 3, 0, 1, 0, 17, 1, 2]
+    L = [9, 3, 21, 16, 0, 40, 1, 18]
+    w = workloads.make_append(seed=30 + policy, n_new=n, seq_lens=L, Hq=8, Hkv=1,
+                              page_size=16, max_pages=3, quant_policy=policy, cos_sin_rows=48,
+                              q_scale_inv=20.0, k_scale=0.05, v_scale=0.05)
+    r, _ = run_and_check(w, schedule=1)
+    assert (r.flags.cpu().numpy() == 0).all()
+
+
 @pytest.mark.parametrize("schedule", SCHEDULES)
 def test_largest_batch(schedule):
     B = 16384
