@@ -655,8 +655,9 @@ def main(argv=None):
                      "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
                      "peak_source": peak_src,
                      "bytes_per_launch": nbytes / args.steps,
-                     "kernel": "fqr::warp_append_kernel<0,0> (latency schedule, chosen "
-                     "automatically)", "timing": "CUDA events around graph "
+                     "kernel": "fqr::warp_append_kernel<0,0,384,true> (latency schedule: "
+                     "12-warp blocks, warp-level batch check; chosen automatically)",
+                     "timing": "CUDA events around graph "
                      "replays of back-to-back launches; average launch = region / steps"},
         "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks, "cpu_baseline": cpu,
         "cpu_baseline_all_cores": cpu_all,

@@ -14,6 +14,8 @@
 //     the second dependent round trip overlaps the batch validation.
 //   * every block stages q_indptr / seq_lens in shared memory and validates the
 //     whole batch (stage_and_validate); a malformed batch writes only flags.
+//     When every warp holds one task and the batch is small, every warp
+//     validates the batch on its own instead (WarpBatchCheck): no barrier.
 //   * the warps of a request's last new row split that request's last-page
 //     tail (both caches) evenly between them and store their share of zeros
 //     before their heads (the stores drain while the heads are computed);
@@ -87,8 +89,18 @@ __device__ __forceinline__ void prefetch_task_lines(const WarpArgs& a, int w, co
   }
 }
 
-template <int POLICY, int STYLE, int NT>
-__global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
+// WV: every warp validates the batch itself (WarpBatchCheck, batches of at
+// most kWarpCheckMaxB requests) and reads metadata and weights from global
+// memory: no block barrier, no shared-memory staging, so no warp waits for
+// the slowest first round trip of its block.  Chosen for launches in which
+// every warp holds one task; correct for any.  Measured on B200 against the
+// block-staged prologue: Qwen3-style decode (128 requests, Hq/Hkv 32/8)
+// 3.82 -> 3.50 us per launch, tiny decode 2.48 -> 2.24 us.
+constexpr int kWarpCheckMaxB = 128;
+constexpr int kWarpCheckMaxPositions = 1024;  // explicit positions: T at most this
+
+template <int POLICY, int STYLE, int NT, bool WV>
+__global__ void __launch_bounds__(NT, NT == kThreads ? 2 : 0) warp_append_kernel(const WarpArgs a) {
   constexpr int NW = NT / 32;  // warps per block
   extern __shared__ __align__(16) int smem[];
   float* s_w = reinterpret_cast<float*>(smem);  // 256 fp32 weights
@@ -171,8 +183,24 @@ __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
   // metadata this thread stages, the norm weights, the first task's packed
   // heads and its own request's metadata (request guessed as b = t: one new
   // row per request, the decode case).
-  const MetaRegs meta = meta_prefetch(a.q_indptr, a.seq_lens, a.B);
-  const WeightRegs<NT> wreg = weight_prefetch_nt<NT>(a.qw, a.kw, a.hp.gemma);
+  const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T,
+               a.B,         a.slot_cap,  a.cs_rows,  a.max_seqlen};
+  MetaRegs meta{0, 0, 0, 0};
+  WeightRegs<NT> wreg;
+  WarpBatchCheck<kWarpCheckMaxB / 32> check;
+  RegWeights wq{make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u), a.hp.gemma};
+  if (WV) {
+    check.load(m, lane);
+    // the lane's own weight slices for its first head (Q or K; none for V)
+    const uint16_t* wsrc = h0 < a.hp.Hq ? a.qw : (h0 < a.hp.Hq + a.hp.Hkv ? a.kw : nullptr);
+    if (own0 && wsrc != nullptr) {
+      wq.wa = __ldg(reinterpret_cast<const uint4*>(wsrc + 8 * l8));
+      wq.wb = __ldg(reinterpret_cast<const uint4*>(wsrc + 64 + 8 * l8));
+    }
+  } else {
+    meta = meta_prefetch(a.q_indptr, a.seq_lens, a.B);
+    wreg = weight_prefetch_nt<NT>(a.qw, a.kw, a.hp.gemma);
+  }
   uint4 pa = make_uint4(0u, 0u, 0u, 0u), pb = pa;
   int e_lo = 0, e_hi = 0, e_L = 0;
   int64_t e_pos = 0;
@@ -209,13 +237,18 @@ __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
         load_cs<STYLE, false>(a.cs + pos * a.hp.rot, a.hp.rot, l8, c0, s0);
     }
   }
-  weight_store_nt<NT>(s_w, wreg);
-  if (a.bulk_tail) zero_buffer_init(s_zero);  // (the prologue's barrier follows)
-  bool issued = false;                        // bulk copies in flight (lane 0)
-
-  const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T,
-               a.B,         a.slot_cap,  a.cs_rows,  a.max_seqlen};
-  if (stage_and_validate(m, s_indptr, s_seq, meta)) return;
+  const bool bulk = !WV && a.bulk_tail;  // (WV: no block-wide zero buffer)
+  bool issued = false;                    // bulk copies in flight (lane 0)
+  if (WV) {
+    const bool bad = check.bad(m, lane);
+    write_flags(m, bad);
+    if (bad) return;
+  } else {
+    weight_store_nt<NT>(s_w, wreg);
+    if (bulk) zero_buffer_init(s_zero);  // (the prologue's barrier follows)
+    if (stage_and_validate(m, s_indptr, s_seq, meta)) return;
+  }
+  const GlobalWeights wg{a.qw, a.kw, a.hp.gemma};
 
   const int n_tasks = a.n_head + a.B;
   for (int w = gwarp; w < n_tasks; w += nwarps) {
@@ -223,7 +256,7 @@ __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
       const uint4 xa = pa, xb = pb;
       if (w + nwarps < a.n_head) {
         warp_load_head(a, w + nwarps, g, l8, pa, pb);
-        prefetch_task_lines(a, w + nwarps, s_indptr, s_seq, lane, paged);
+        if (!WV) prefetch_task_lines(a, w + nwarps, s_indptr, s_seq, lane, paged);
       }
       const int t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
       const int quad = w - t * a.quads;
@@ -231,45 +264,57 @@ __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
         // (the tail stores need nothing from the head: issue them first so they
         // drain while the head is computed)
         if (paged && r0.is_last && !a.own_tails) {
-          if (a.bulk_tail)
+          if (bulk)
             issued |= zero_tail_share_bulk(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane, s_zero);
           else
             zero_tail_share(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane);
         }
-        process_quad_cs<POLICY, STYLE>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, s_w, l8, gmask);
+        if (WV)
+          process_quad_cs<POLICY, STYLE>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, wq, l8,
+                                         gmask);
+        else
+          process_quad_cs<POLICY, STYLE>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, s_w, l8,
+                                         gmask);
         continue;
       }
       const int h = quad * 4 + g;
-      const int b = request_of_row(s_indptr, a.B, t);
-      const int end = s_indptr[b + 1];
-      const int p_slot = t + s_seq[b] - end;
+      const int b = WV ? request_of_row_global(a.q_indptr, a.B, t) : request_of_row(s_indptr, a.B, t);
+      const int beg = WV ? __ldg(a.q_indptr + b) : s_indptr[b];
+      const int end = WV ? __ldg(a.q_indptr + b + 1) : s_indptr[b + 1];
+      const int p_slot = t + (WV ? __ldg(a.seq_lens + b) : s_seq[b]) - end;
       const int pidx = static_cast<int>(a.hp.pdiv.div(static_cast<uint32_t>(p_slot)));
       RowCtx r;
       r.t = t;
       r.slot_row = p_slot - pidx * a.hp.page_size;
       r.pos = a.positions != nullptr ? static_cast<int>(a.positions[t]) : p_slot;
       r.is_last = t == end - 1;
-      r.qs = q_scale_row(a.hp, t, b, t - s_indptr[b]);
+      r.qs = q_scale_row(a.hp, t, b, t - beg);
       const bool share = paged && r.is_last && !a.own_tails;
       r.page = paged && (h >= a.hp.Hq || share)
                    ? __ldg(a.page_table + static_cast<int64_t>(b) * a.max_pages + pidx)
                    : 0;
       if (share) {
-        if (a.bulk_tail)
+        if (bulk)
           issued |= zero_tail_share_bulk(a.hp, r.page, r.slot_row, quad, a.qdiv, lane, s_zero);
         else
           zero_tail_share(a.hp, r.page, r.slot_row, quad, a.qdiv, lane);
       }
       // (a group past the last head only helps with the tail)
       const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
-      process_quad<POLICY, STYLE, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, s_w, l8,
-                                         gmask);
+      if (WV)
+        process_quad<POLICY, STYLE, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, wg, l8,
+                                           gmask);
+      else
+        process_quad<POLICY, STYLE, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, s_w, l8,
+                                           gmask);
     } else {
       // request task: the tail of a request without new rows (whose tail no
       // head task shares), or of every request when request tasks own tails
       const int b = w - a.n_head;
-      const int L = s_seq[b];
-      if (paged && L > 0 && (a.own_tails || s_indptr[b] == s_indptr[b + 1]))
+      const int L = WV ? __ldg(a.seq_lens + b) : s_seq[b];
+      const bool empty = WV ? __ldg(a.q_indptr + b) == __ldg(a.q_indptr + b + 1)
+                            : s_indptr[b] == s_indptr[b + 1];
+      if (paged && L > 0 && (a.own_tails || empty))
         zero_request_tail<POLICY == 0 ? 2 : 1>(a.hp, a.page_table, a.max_pages, b, L, lane);
     }
   }
@@ -278,21 +323,24 @@ __global__ void __launch_bounds__(NT) warp_append_kernel(const WarpArgs a) {
 
 using WarpKernel = void (*)(const WarpArgs);
 
-template <int NT>
+template <int NT, bool WV>
 static WarpKernel select_warp_nt(int policy, int style) {
   if (style == 0) {
-    if (policy == 0) return warp_append_kernel<0, 0, NT>;
-    if (policy == 1) return warp_append_kernel<1, 0, NT>;
-    return warp_append_kernel<2, 0, NT>;
+    if (policy == 0) return warp_append_kernel<0, 0, NT, WV>;
+    if (policy == 1) return warp_append_kernel<1, 0, NT, WV>;
+    return warp_append_kernel<2, 0, NT, WV>;
   }
-  if (policy == 0) return warp_append_kernel<0, 1, NT>;
-  if (policy == 1) return warp_append_kernel<1, 1, NT>;
-  return warp_append_kernel<2, 1, NT>;
+  if (policy == 0) return warp_append_kernel<0, 1, NT, WV>;
+  if (policy == 1) return warp_append_kernel<1, 1, NT, WV>;
+  return warp_append_kernel<2, 1, NT, WV>;
 }
 
-static WarpKernel select_warp(int policy, int style, int nt) {
-  return nt == kWideThreads ? select_warp_nt<kWideThreads>(policy, style)
-                            : select_warp_nt<kThreads>(policy, style);
+static WarpKernel select_warp(int policy, int style, int nt, bool wv = false) {
+  if (wv)
+    return nt == kWideThreads ? select_warp_nt<kWideThreads, true>(policy, style)
+                              : select_warp_nt<kThreads, true>(policy, style);
+  return nt == kWideThreads ? select_warp_nt<kWideThreads, false>(policy, style)
+                            : select_warp_nt<kThreads, false>(policy, style);
 }
 
 static size_t warp_smem(const fqr_append_params& p) {
@@ -309,19 +357,17 @@ int64_t latency_tasks(const fqr_append_params& p) {
 // per SM holds every task, the wide block spreads the warps evenly: an SM
 // with twice the warps of its neighbours takes longer in every phase of the
 // launch (load round trips, prologue, stores), and it sets the launch time.
-// Measured on B200 (paged BF16 decode, Hq/Hkv 32/8, page 16, 128 requests:
-// 1,664 warp tasks): 4.04 us per launch with 208 blocks of 8 warps (60 SMs
-// with 16 warps), 3.81 us with 139 blocks of 12.  Without request tails
-// (caller-owned K/V) the launch is short enough that the wide block's lost
-// residency overlap costs more than it gains, so those keep kThreads.
+// Measured on B200 (decode, Hq/Hkv 32/8, 128 requests: 1,664 warp tasks;
+// 208 blocks of 8 warps leave 60 SMs with 16 warps, 139 blocks of 12 one
+// per SM): paged K/V 3.55 -> 3.49 us per launch, caller-owned K/V 3.01 ->
+// 2.91 us (with the warp-level batch check; 4.04 -> 3.81 us before it).
 int warp_block_threads(const fqr_append_params& p) {
   DeviceInfo d;
   if (device_info(&d) != FQR_OK) return kThreads;
   const int64_t tasks = latency_tasks(p);
   const int64_t narrow_blocks = (tasks + kWarps - 1) / kWarps;
   const int64_t wide_blocks = (tasks + kWideThreads / 32 - 1) / (kWideThreads / 32);
-  const bool paged = p.out_k == nullptr;
-  return paged && narrow_blocks > d.sms && wide_blocks <= d.sms ? kWideThreads : kThreads;
+  return narrow_blocks > d.sms && wide_blocks <= d.sms ? kWideThreads : kThreads;
 }
 
 int64_t latency_capacity(const fqr_append_params& p) {
@@ -371,7 +417,12 @@ int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStr
   a.flags = p.flags;
   const size_t smem = warp_smem(p);
   const int nt = warp_block_threads(p);
-  WarpKernel k = select_warp(p.quant_policy, p.rope_style, nt);
+  // Warp-level validation when every warp holds one task (the launch is one
+  // pass) and the batch is small enough for one warp to check.
+  const int64_t cap = latency_capacity(p);
+  const bool wv = cap >= n_head + p.B && p.B <= kWarpCheckMaxB &&
+                  (p.positions == nullptr || p.T <= kWarpCheckMaxPositions);
+  WarpKernel k = select_warp(p.quant_policy, p.rope_style, nt, wv);
   return launch_persistent(
       reinterpret_cast<const void*>(k), n_head + p.B, smem, stream,
       [&](int grid) {

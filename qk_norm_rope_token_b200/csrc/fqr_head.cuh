@@ -139,6 +139,57 @@ __device__ __forceinline__ void unpack_pairs(uint4 xa, uint4 xb, float2* y) {
   y[7] = make_float2(bf16_lo(xb.w), bf16_hi(xb.w));
 }
 
+// Norm-weight sources of the head arithmetic (load_weights): the block's
+// staged fp32 copy (a `const float*` filled by weight_store), the lane's two
+// 16-byte slices of the BF16 weight vector already in registers (RegWeights:
+// wa = elements [8l, 8l+8), wb = [64+8l, 64+8l+8), loaded in a task's first
+// round trip), or those slices read from global memory at the norm
+// (GlobalWeights).  The last two need no block-wide staging.
+struct RegWeights {
+  uint4 wa, wb;
+  int gemma;
+};
+struct GlobalWeights {
+  const uint16_t* qw;
+  const uint16_t* kw;
+  int gemma;
+};
+
+__device__ __forceinline__ void load_weights(const float* s_w, bool is_q, int l8, float2* w) {
+  const float* wv = s_w + (is_q ? 0 : kHeadDim) + 4 * l8;
+  const float4 w0 = lds_f4(wv);
+  const float4 w1 = lds_f4(wv + 32);
+  const float4 w2 = lds_f4(wv + 64);
+  const float4 w3 = lds_f4(wv + 96);
+  w[0] = make_float2(w0.x, w0.y);
+  w[1] = make_float2(w0.z, w0.w);
+  w[2] = make_float2(w1.x, w1.y);
+  w[3] = make_float2(w1.z, w1.w);
+  w[4] = make_float2(w2.x, w2.y);
+  w[5] = make_float2(w2.z, w2.w);
+  w[6] = make_float2(w3.x, w3.y);
+  w[7] = make_float2(w3.z, w3.w);
+}
+// BF16 slices -> the lane's 8 weight pairs; the Gemma-style norm scales by
+// 1 + w, formed in fp32 exactly as weight_value forms it.
+__device__ __forceinline__ void unpack_weights(uint4 wa, uint4 wb, int gemma, float2* w) {
+  unpack_pairs(wa, wb, w);
+  if (gemma) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = __fadd2_rn(make_float2(1.0f, 1.0f), w[j]);
+  }
+}
+__device__ __forceinline__ void load_weights(const RegWeights& r, bool /*is_q*/, int /*l8*/,
+                                             float2* w) {
+  unpack_weights(r.wa, r.wb, r.gemma, w);
+}
+__device__ __forceinline__ void load_weights(const GlobalWeights& g, bool is_q, int l8,
+                                             float2* w) {
+  const uint16_t* src = is_q ? g.qw : g.kw;
+  unpack_weights(__ldg(reinterpret_cast<const uint4*>(src + 8 * l8)),
+                 __ldg(reinterpret_cast<const uint4*>(src + 64 + 8 * l8)), g.gemma, w);
+}
+
 __device__ __forceinline__ uint4 pack_bf16_pairs(const float2* y) {
   return make_uint4(pack_bf16x2(y[0].x, y[0].y), pack_bf16x2(y[1].x, y[1].y),
                     pack_bf16x2(y[2].x, y[2].y), pack_bf16x2(y[3].x, y[3].y));
@@ -319,13 +370,14 @@ __device__ __forceinline__ int quad_kind(const HeadParams& a, int h0) {
 
 // Norm + RoPE + quantisation + store of head h of row r.  xa/xb: the lane's two
 // 16-byte slices of the packed head; cs_row: the row's fp32 [cos | sin]
-// (shared or global memory); s_w: staged weights.  gmask: the 8-lane group.
-// KIND: the head's kind when the caller knows it (HeadKind).  Request tails
-// are zeroed by the callers (zero_tail_share), not here.
-template <int POLICY, int STYLE, int KIND = kAnyHead>
+// (shared or global memory); wts: the norm weights (load_weights).  gmask:
+// the 8-lane group.  KIND: the head's kind when the caller knows it
+// (HeadKind).  Request tails are zeroed by the callers (zero_tail_share), not
+// here.
+template <int POLICY, int STYLE, int KIND = kAnyHead, class W>
 __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCtx& r, int h,
                                                 uint4 xa, uint4 xb, const float2* c,
-                                                const float2* s, const float* s_w, int l8,
+                                                const float2* s, const W& wts, int l8,
                                                 unsigned gmask) {
   constexpr int ES = POLICY == 0 ? 2 : 1;
   float2 y[8];
@@ -363,15 +415,8 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
     // the parity bar propagates the difference with that of the summation order
     const float inv = rsqrtf(__fadd_rn(ss * (1.0f / kHeadDim), a.eps));
     const float2 iv = make_float2(inv, inv);
-    const float* wv = s_w + (is_q ? 0 : kHeadDim) + 4 * l8;
-    const float4 w0 = lds_f4(wv);
-    const float4 w1 = lds_f4(wv + 32);
-    const float4 w2 = lds_f4(wv + 64);
-    const float4 w3 = lds_f4(wv + 96);
-    const float2 w[8] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w),
-                         make_float2(w1.x, w1.y), make_float2(w1.z, w1.w),
-                         make_float2(w2.x, w2.y), make_float2(w2.z, w2.w),
-                         make_float2(w3.x, w3.y), make_float2(w3.z, w3.w)};
+    float2 w[8];
+    load_weights(wts, is_q, l8, w);
 #pragma unroll
     for (int j = 0; j < 8; ++j) y[j] = mul2(mul2(y[j], iv), w[j]);
   }
@@ -431,53 +476,53 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
 
 // As process_head_cs, loading the cos/sin values from cs_row first (V heads
 // need none).
-template <int POLICY, int STYLE, bool CS_SMEM, int KIND = kAnyHead>
+template <int POLICY, int STYLE, bool CS_SMEM, int KIND = kAnyHead, class W>
 __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& r, int h,
                                              uint4 xa, uint4 xb, const float* cs_row,
-                                             const float* s_w, int l8, unsigned gmask) {
+                                             const W& wts, int l8, unsigned gmask) {
   float2 c[4], s[4];
   if (KIND == kQHead || KIND == kKHead || (KIND == kAnyHead && h < a.Hq + a.Hkv))
     load_cs<STYLE, CS_SMEM>(cs_row, a.rot, l8, c, s);
-  process_head_cs<POLICY, STYLE, KIND>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+  process_head_cs<POLICY, STYLE, KIND>(a, r, h, xa, xb, c, s, wts, l8, gmask);
 }
 
 // process_head_cs for one quad whose first head is h0 (warp-uniform), with
 // the cos/sin values already loaded; see process_quad.
-template <int POLICY, int STYLE>
+template <int POLICY, int STYLE, class W>
 __device__ __forceinline__ void process_quad_cs(const HeadParams& a, const RowCtx& r, int h0,
                                                 int nheads, int g, uint4 xa, uint4 xb,
-                                                const float2* c, const float2* s,
-                                                const float* s_w, int l8, unsigned gmask) {
+                                                const float2* c, const float2* s, const W& wts,
+                                                int l8, unsigned gmask) {
   const int h = h0 + g;
   const int kind = h0 + 4 <= nheads ? quad_kind(a, h0) : kAnyHead;
   if (kind == kQHead)
-    process_head_cs<POLICY, STYLE, kQHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+    process_head_cs<POLICY, STYLE, kQHead>(a, r, h, xa, xb, c, s, wts, l8, gmask);
   else if (kind == kKHead)
-    process_head_cs<POLICY, STYLE, kKHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+    process_head_cs<POLICY, STYLE, kKHead>(a, r, h, xa, xb, c, s, wts, l8, gmask);
   else if (kind == kVHead)
-    process_head_cs<POLICY, STYLE, kVHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+    process_head_cs<POLICY, STYLE, kVHead>(a, r, h, xa, xb, c, s, wts, l8, gmask);
   else if (h < nheads)
-    process_head_cs<POLICY, STYLE, kAnyHead>(a, r, h, xa, xb, c, s, s_w, l8, gmask);
+    process_head_cs<POLICY, STYLE, kAnyHead>(a, r, h, xa, xb, c, s, wts, l8, gmask);
 }
 
 // process_head for one quad whose first head is h0 (warp-uniform): the kind
 // is decided once for the warp when all four heads exist; otherwise each
 // group decides for its own head (h0 + g < nheads).
-template <int POLICY, int STYLE, bool CS_SMEM>
+template <int POLICY, int STYLE, bool CS_SMEM, class W>
 __device__ __forceinline__ void process_quad(const HeadParams& a, const RowCtx& r, int h0,
                                              int nheads, int g, uint4 xa, uint4 xb,
-                                             const float* cs_row, const float* s_w, int l8,
+                                             const float* cs_row, const W& wts, int l8,
                                              unsigned gmask) {
   const int h = h0 + g;
   const int kind = h0 + 4 <= nheads ? quad_kind(a, h0) : kAnyHead;
   if (kind == kQHead)
-    process_head<POLICY, STYLE, CS_SMEM, kQHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kQHead>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
   else if (kind == kKHead)
-    process_head<POLICY, STYLE, CS_SMEM, kKHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kKHead>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
   else if (kind == kVHead)
-    process_head<POLICY, STYLE, CS_SMEM, kVHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kVHead>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
   else if (h < nheads)
-    process_head<POLICY, STYLE, CS_SMEM, kAnyHead>(a, r, h, xa, xb, cs_row, s_w, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kAnyHead>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
 }
 
 // Zero the whole tail (rows [last+1, P), all heads) of request b's last page in
