@@ -96,8 +96,6 @@ __device__ __forceinline__ void prefetch_task_lines(const WarpArgs& a, int w, co
 // every warp holds one task; correct for any.  Measured on B200 against the
 // block-staged prologue: Qwen3-style decode (128 requests, Hq/Hkv 32/8)
 // 3.82 -> 3.50 us per launch, tiny decode 2.48 -> 2.24 us.
-constexpr int kWarpCheckMaxB = 128;
-constexpr int kWarpCheckMaxPositions = 1024;  // explicit positions: T at most this
 
 template <int POLICY, int STYLE, int NT, bool WV>
 __global__ void __launch_bounds__(NT, NT == kThreads ? 2 : 0) warp_append_kernel(const WarpArgs a) {
