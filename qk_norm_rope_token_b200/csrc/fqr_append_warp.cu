@@ -148,10 +148,15 @@ __global__ void __launch_bounds__(NT, NT == kThreads ? 2 : 0) warp_append_kernel
       }
       // ... and, from a possibly stale read of that metadata (L2 only), the
       // lines of the second round trip: the page-table entry and the cos/sin
-      // row (a wrong guess costs only a useless prefetch)
+      // row (a wrong guess costs only a useless prefetch).  Only for paged
+      // K/V: the read's latency delays the warp's arrival at the dependency
+      // wait, which a cos/sin row alone does not repay (measured on B200,
+      // decode into caller-owned K/V, 128 requests, Hq/Hkv 32/8: 2.90 ->
+      // 2.75 us per launch without it; the paged Qwen3-style decode loses
+      // 3.48 -> 3.55 us without it).
       int lo = 0, hi = 0, L = 0;
       int64_t ps = 0;
-      if (lane == 0) {
+      if (lane == 0 && paged) {
         lo = ld_cg_s32(a.q_indptr + gb);
         hi = ld_cg_s32(a.q_indptr + gb + 1);
         L = ld_cg_s32(a.seq_lens + gb);
