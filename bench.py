@@ -89,10 +89,16 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
 
 
-def kernel_source_hash() -> str:
+# The sources the fused append's kernels are built from (the MLA kernels, the
+# host entry points and the runtime are not among them).
+APPEND_KERNEL_SOURCES = ("fqr_append.cu", "fqr_append_pipe.cu", "fqr_append_warp.cu",
+                         "fqr_device.cuh", "fqr_head.cuh", "fqr_launch.h")
+
+
+def kernel_source_hash(names=APPEND_KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "qk_norm_rope_token_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(names):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
