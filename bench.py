@@ -79,6 +79,22 @@ def parse_args(argv=None):
 
 # ------------------------------------------------------------------ helpers
 
+def describe_plan(plan: dict) -> str:
+    """The launch fqr_append_plan_query reports, in words."""
+    if plan["schedule"] == 2:
+        return (f"fqr::pipe_append_kernel (streaming schedule: {plan['grid']} blocks of "
+                f"{plan['block_threads']} threads, {plan['tasks']} units; chosen automatically)")
+    extra = [("warp-level batch check" if plan["warp_check"] else "block batch prologue"),
+             "quad-major head tasks"]
+    if plan["bulk_tails"]:
+        extra.append("bulk-copy tails")
+    if plan["request_tails"]:
+        extra.append("request tasks own the tails")
+    return (f"fqr::warp_append_kernel (latency schedule: {plan['grid']} blocks of "
+            f"{plan['block_threads']} threads, {plan['tasks']} warp tasks, " + ", ".join(extra) +
+            "; chosen automatically)")
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -661,8 +677,7 @@ def main(argv=None):
                      "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
                      "peak_source": peak_src,
                      "bytes_per_launch": nbytes / args.steps,
-                     "kernel": "fqr::warp_append_kernel<0,0,384,true> (latency schedule: "
-                     "12-warp blocks, warp-level batch check; chosen automatically)",
+                     "kernel": describe_plan(fqr.append_plan(bench.reps[0]["params"])),
                      "timing": "CUDA events around graph "
                      "replays of back-to-back launches; average launch = region / steps"},
         "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks, "cpu_baseline": cpu,

@@ -178,6 +178,43 @@ typedef struct fqr_append_params {
 int fqr_append_paged(const fqr_append_params* p, void* stream);
 
 /*
+ * fqr_append_plan_query -- the launch fqr_append_paged would make for *p on
+ * the current device, without making it: which schedule, the grid and block
+ * shape, and the variants of the latency schedule.  The FlashInfer PR #5956
+ * wrapper exposes its launch plan the same way ("launch_plan"); this is its
+ * counterpart, for callers that size or log their launches and for tests.
+ *
+ *   schedule       FQR_SCHEDULE_LATENCY or FQR_SCHEDULE_STREAMING; 0 when the
+ *                  call would launch nothing (T = B = 0).
+ *   grid           blocks of the launch.
+ *   block_threads  threads per block.
+ *   tasks          latency: warp tasks (a quad of heads of a row, or a
+ *                  request's tail); streaming: units (a packed row, or a
+ *                  chunk of one).
+ *   warp_check     latency: every warp validates the batch itself (no block
+ *                  prologue); streaming: 0.
+ *   bulk_tails     latency: tails go out as bulk copies (warps hold several
+ *                  tasks).
+ *   request_tails  latency: request tasks zero whole tails (small tails, one
+ *                  task per warp).
+ *
+ * Checks *p exactly as fqr_append_paged does and returns the same codes;
+ * `plan` must not be NULL (FQR_EINVAL).  Queries the device (SM count,
+ * occupancy; cached per device after the first call); launches, allocates
+ * and synchronises nothing.
+ */
+typedef struct fqr_append_plan {
+  int32_t schedule;
+  int32_t grid;
+  int32_t block_threads;
+  int32_t tasks;
+  int32_t warp_check;
+  int32_t bulk_tails;
+  int32_t request_tails;
+} fqr_append_plan;
+int fqr_append_plan_query(const fqr_append_params* p, fqr_append_plan* plan);
+
+/*
  * fqr_pipeline_* -- fqr_append_paged on batches held in pinned host memory,
  * pipelined.  A pipeline has `depth` slots; slot j owns a device input buffer
  * dev_in[j] (in_bytes) and a device result buffer dev_out[j] (out_bytes),

@@ -51,6 +51,12 @@ class AppendParams(ctypes.Structure):
     ]
 
 
+class AppendPlan(ctypes.Structure):
+    """Mirror of fqr_append_plan."""
+    _fields_ = [("schedule", c_i32), ("grid", c_i32), ("block_threads", c_i32), ("tasks", c_i32),
+                ("warp_check", c_i32), ("bulk_tails", c_i32), ("request_tails", c_i32)]
+
+
 class MlaParams(ctypes.Structure):
     """Mirror of fqr_mla_params."""
     _fields_ = [
@@ -78,6 +84,9 @@ def _load() -> ctypes.CDLL:
     lib.fqr_append_paged.restype = ctypes.c_int
     lib.fqr_concat_mla_cache.argtypes = [ctypes.POINTER(MlaParams), c_vp]
     lib.fqr_concat_mla_cache.restype = ctypes.c_int
+    lib.fqr_append_plan_query.argtypes = [ctypes.POINTER(AppendParams),
+                                          ctypes.POINTER(AppendPlan)]
+    lib.fqr_append_plan_query.restype = ctypes.c_int
     lib.fqr_strerror.argtypes = [ctypes.c_int]
     lib.fqr_strerror.restype = ctypes.c_char_p
     lib.fqr_pipeline_create.argtypes = [ctypes.c_int, ctypes.POINTER(AppendParams),
@@ -111,6 +120,17 @@ def strerror(code: int) -> str:
 def append_paged_raw(params: AppendParams, stream: int = 0) -> int:
     """Call fqr_append_paged with a filled parameter struct; returns the code."""
     return LIB.fqr_append_paged(ctypes.byref(params), c_vp(stream))
+
+
+def append_plan(params: AppendParams) -> dict:
+    """fqr_append_plan_query: the launch fqr_append_paged would make for these
+    parameters on the current device (nothing is launched).  Raises FqrError
+    on a rejected argument."""
+    plan = AppendPlan()
+    rc = LIB.fqr_append_plan_query(ctypes.byref(params), ctypes.byref(plan))
+    if rc != FQR_OK:
+        raise FqrError(rc)
+    return {name: int(getattr(plan, name)) for name, _ in AppendPlan._fields_}
 
 
 def concat_mla_cache_raw(params: MlaParams, stream: int = 0) -> int:

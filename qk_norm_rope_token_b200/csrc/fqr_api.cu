@@ -142,6 +142,15 @@ int fqr_append_paged(const fqr_append_params* p, void* stream) {
   return fqr::launch_append(*p, static_cast<cudaStream_t>(stream));
 }
 
+int fqr_append_plan_query(const fqr_append_params* p, fqr_append_plan* plan) {
+  if (plan == nullptr) return FQR_EINVAL;
+  *plan = fqr_append_plan{0, 0, 0, 0, 0, 0, 0};
+  if (p != nullptr && p->T == 0 && p->B == 0) return FQR_OK;  // nothing would launch
+  const int rc = fqr::check_append(p);
+  if (rc != FQR_OK) return rc;
+  return fqr::launch_append(*p, nullptr, plan);
+}
+
 int fqr_concat_mla_cache(const fqr_mla_params* p, void* stream) {
   if (p != nullptr && p->T == 0 && p->B == 0) return FQR_OK;
   const int rc = check_mla(p);

@@ -16,7 +16,7 @@ namespace fqr {
 constexpr int64_t kLargeTail = 48 * 1024;  // expected tail bytes per row (both caches)
 constexpr int64_t kLargeTailPasses = 8;
 
-int launch_append(const fqr_append_params& p, cudaStream_t stream) {
+int launch_append(const fqr_append_params& p, cudaStream_t stream, fqr_append_plan* plan) {
   HeadParams hp;
   const int es = p.quant_policy == 0 ? 2 : 1;
   const bool owned = p.out_k != nullptr;
@@ -69,8 +69,8 @@ int launch_append(const fqr_append_params& p, cudaStream_t stream) {
                    ? FQR_SCHEDULE_LATENCY
                    : FQR_SCHEDULE_STREAMING;
   }
-  return schedule == FQR_SCHEDULE_STREAMING ? launch_append_pipe(p, hp, stream)
-                                            : launch_append_warp(p, hp, stream);
+  return schedule == FQR_SCHEDULE_STREAMING ? launch_append_pipe(p, hp, stream, plan)
+                                            : launch_append_warp(p, hp, stream, plan);
 }
 
 }  // namespace fqr

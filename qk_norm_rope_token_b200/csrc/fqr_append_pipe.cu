@@ -368,7 +368,8 @@ static PipeKernel select_pipe(int policy, int style) {
   return pipe_append_kernel<2, 1>;
 }
 
-int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream) {
+int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream,
+                       fqr_append_plan* plan) {
   PipeArgs a;
   a.hp = hp;
   a.qkv = p.qkv;
@@ -427,6 +428,11 @@ int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStr
   const int64_t cap = static_cast<int64_t>(per_sm) * sms;
   const int64_t want = a.units > sms ? a.units : sms;
   const int grid = static_cast<int>(want < cap ? want : cap);
+  if (plan != nullptr) {
+    *plan = fqr_append_plan{FQR_SCHEDULE_STREAMING, grid, kPipeThreads, static_cast<int32_t>(a.units),
+                            0, 0, 0};
+    return FQR_OK;
+  }
   return launch_pdl(k, grid, kPipeThreads, smem, stream, a);
 }
 

@@ -413,7 +413,8 @@ int64_t latency_capacity(const fqr_append_params& p) {
 // 3.57 us at 4 requests with whole tails, so those keep the shares.
 constexpr int64_t kOwnTailsMaxBytes = 4096;
 
-int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream) {
+int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream,
+                       fqr_append_plan* plan) {
   WarpArgs a;
   a.hp = hp;
   a.qkv = p.qkv;
@@ -460,6 +461,11 @@ int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStr
         a.bulk_tail = static_cast<int64_t>(grid) * (nt / 32) < n_head + p.B;
         a.own_tails = !a.bulk_tail && static_cast<int64_t>(p.page_size - 1) * hp.row_bytes <=
                                           kOwnTailsMaxBytes;
+        if (plan != nullptr) {
+          *plan = fqr_append_plan{FQR_SCHEDULE_LATENCY, grid, nt, a.n_head + p.B, wv ? 1 : 0,
+                                  a.bulk_tail, a.own_tails};
+          return FQR_OK;
+        }
         return launch_pdl(k, grid, nt, smem, stream, a);
       },
       nt);

@@ -13,15 +13,20 @@ namespace fqr {
 struct HeadParams;
 // Host-side argument checks of fqr_append_paged (FQR_OK or the error code).
 int check_append(const fqr_append_params* p);
-int launch_append(const fqr_append_params& p, cudaStream_t stream);
-int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream);
+// The launch of fqr_append_paged on `stream`; with `plan` non-null, the plan
+// of that launch instead (nothing is launched).
+int launch_append(const fqr_append_params& p, cudaStream_t stream,
+                  fqr_append_plan* plan = nullptr);
+int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream,
+                       fqr_append_plan* plan = nullptr);
 // Warp tasks of the latency schedule for p, and how many warps of it the
 // device holds at once (-1 if the runtime cannot tell).
 int64_t latency_tasks(const fqr_append_params& p);
 int64_t latency_capacity(const fqr_append_params& p);
 // Threads per block the latency schedule uses for p (fqr_append_warp.cu).
 int warp_block_threads(const fqr_append_params& p);
-int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream);
+int launch_append_pipe(const fqr_append_params& p, const HeadParams& hp, cudaStream_t stream,
+                       fqr_append_plan* plan = nullptr);
 int launch_mla(const fqr_mla_params& p, cudaStream_t stream);
 
 // Launch facts of the current device, cached after the first query

@@ -199,6 +199,14 @@ class AppendRun:
                          None if nul else self.v_cache, self.out_q, self.flags, stream=stream,
                          **self.kwargs())
 
+    def plan(self):
+        """The launch plan of this call (fqr_append_plan_query)."""
+        nul = self.null_caches
+        return fqr.append_plan(fqr.append_params(
+            self.qkv, self.cs, self.indptr_d, self.seq_d, None if nul else self.pt_d,
+            None if nul else self.k_cache, None if nul else self.v_cache, self.out_q, self.flags,
+            **self.kwargs()))
+
     # ------------------------------------------------------------ checking --
     def run_oracle(self):
         w = self.w

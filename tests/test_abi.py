@@ -32,7 +32,8 @@ def declared_functions():
 
 
 def test_header_declares_the_entry_points():
-    assert declared_functions() == ["fqr_append_paged", "fqr_concat_mla_cache",
+    assert declared_functions() == ["fqr_append_paged", "fqr_append_plan_query",
+                                    "fqr_concat_mla_cache",
                                     "fqr_pipeline_create", "fqr_pipeline_destroy",
                                     "fqr_pipeline_fork", "fqr_pipeline_join",
                                     "fqr_pipeline_submit", "fqr_pipeline_sync", "fqr_strerror"]
@@ -48,11 +49,12 @@ def test_library_exports_every_declared_symbol(fqr):
     assert set(declared_functions()) <= exported
 
 
-@pytest.mark.parametrize("struct", ["fqr_append_params", "fqr_mla_params"])
+@pytest.mark.parametrize("struct", ["fqr_append_params", "fqr_mla_params", "fqr_append_plan"])
 def test_struct_layout_matches_binding(fqr, struct, tmp_path):
     """Compile a probe against the header and compare sizeof / offsetof of
     every field with the ctypes mirror."""
-    cls = fqr.AppendParams if struct == "fqr_append_params" else fqr.MlaParams
+    cls = {"fqr_append_params": fqr.AppendParams, "fqr_mla_params": fqr.MlaParams,
+           "fqr_append_plan": fqr.AppendPlan}[struct]
     fields = [f for f, _ in cls._fields_]
     src = tmp_path / "probe.c"
     body = "".join(f'printf("{f} %zu\\n", offsetof({struct}, {f}));\n' for f in fields)
@@ -163,6 +165,28 @@ def test_append_owned_kv_needs_no_cache_or_page_table(fqr):
     for over in (OWNED_OK, dict(OWNED_OK, norm_style=1),
                  dict(quant_policy=1, q_scale=FAKE, k_scale=FAKE, v_scale=FAKE, max_seqlen=129)):
         assert fqr.append_paged_raw(valid_append(fqr, **over)) == fqr.FQR_ECUDA
+
+
+def test_plan_query_checks_like_the_call(fqr):
+    """fqr_append_plan_query applies fqr_append_paged's host checks, returns
+    their codes, and answers an empty batch without touching the device."""
+    plan = fqr.AppendPlan()
+    assert fqr.LIB.fqr_append_plan_query(ctypes.byref(valid_append(fqr)), None) == fqr.FQR_EINVAL
+    for case in sorted(APPEND_BAD):
+        rc = fqr.LIB.fqr_append_plan_query(ctypes.byref(valid_append(fqr, **APPEND_BAD[case])),
+                                           ctypes.byref(plan))
+        assert rc == fqr.FQR_EINVAL, case
+    assert fqr.LIB.fqr_append_plan_query(ctypes.byref(valid_append(fqr, rot_dim=64)),
+                                         ctypes.byref(plan)) == fqr.FQR_ENOTSUP
+    p = valid_append(fqr, T=0, B=0, qkv=None, out_q=None, q_indptr=None, seq_lens=None,
+                     page_table=None, flags=None)
+    plan.grid = 7
+    assert fqr.LIB.fqr_append_plan_query(ctypes.byref(p), ctypes.byref(plan)) == fqr.FQR_OK
+    assert (plan.schedule, plan.grid, plan.block_threads, plan.tasks) == (0, 0, 0, 0)
+    # valid parameters need the device's occupancy: on a machine without a GPU
+    # the query reaches the CUDA runtime and reports that
+    assert fqr.LIB.fqr_append_plan_query(ctypes.byref(valid_append(fqr)),
+                                         ctypes.byref(plan)) == fqr.FQR_ECUDA
 
 
 def test_append_null_params(fqr):

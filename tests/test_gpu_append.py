@@ -157,6 +157,31 @@ def test_wide_block_preconditions_hold_on_this_device():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     tasks = 128 * 12 + 128
     assert -(-tasks // 8) > sms and -(-tasks // 12) <= sms, sms
+    plan = AppendRun(_wide_block_decode(0, 0), schedule=0).plan()
+    assert plan["schedule"] == 1 and plan["block_threads"] == 384 and plan["warp_check"] == 1
+
+
+# The launch plans of the named workloads on a 148-SM B200: which schedule and
+# which latency-schedule variants the parity tests above exercise.
+PLANS = {
+    "qwen3_decode_bf16": dict(schedule=1, block_threads=384, grid=139, tasks=1664, warp_check=1,
+                              bulk_tails=0, request_tails=0),
+    "tiny_decode_bf16": dict(schedule=1, block_threads=256, grid=2, tasks=16, warp_check=1,
+                             bulk_tails=0, request_tails=1),
+    "fp8_decode_dynamic": dict(schedule=1, block_threads=256, tasks=5376, warp_check=0,
+                               bulk_tails=1, request_tails=0),
+    "decode_out_kv_bf16": dict(schedule=1, block_threads=384, warp_check=1),
+    "ragged_prefill_fp8": dict(schedule=2, block_threads=288, warp_check=0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PLANS))
+def test_launch_plan_of_named_workloads(name):
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("plans recorded for a 148-SM B200")
+    plan = AppendRun(workloads.APPEND_CONFIGS[name](), schedule=0).plan()
+    for k, v in PLANS[name].items():
+        assert plan[k] == v, (k, plan)
 
 
 @pytest.mark.parametrize("style", [0, 1])
