@@ -43,19 +43,25 @@ int resident_blocks(const void* fn, int threads, size_t smem, int* per_sm);
 // Launch `kernel(args)` on `stream` with programmatic stream serialization,
 // so that it may begin while the preceding kernel in the stream finishes; the
 // kernel itself waits (griddepcontrol.wait) before reading any input.
+// cluster > 1: the grid is launched as thread-block clusters of that many
+// blocks (grid a multiple of it).
 template <class Args>
 int launch_pdl(void (*kernel)(const Args), int grid, int threads, size_t smem,
-               cudaStream_t stream, const Args& args) {
+               cudaStream_t stream, const Args& args, int cluster = 1) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(static_cast<unsigned>(threads));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
   if (cudaLaunchKernelEx(&cfg, kernel, args) != cudaSuccess) {
     (void)cudaGetLastError();
     return FQR_ECUDA;

@@ -15,9 +15,12 @@
 //     covers the NeoX pairs (i, i+32) and the GPT-J pairs (2i, 2i+1) alike.
 // With Q quantisation the 8 lanes of a head also hold its nope part in
 // 16-byte chunks: static and per-head scales keep the warp tasks
-// (mla_quant_kernel); per-token scales give a block of up to 32 warps a whole
-// row of Q at a time (mla_token_kernel), its maximum reduced over the block
-// before any payload store.
+// (mla_quant_kernel); per-token scales give a thread-block cluster of
+// kTokenCluster blocks a whole row of Q at a time (mla_token_kernel), its
+// maximum reduced over the cluster (distributed shared memory) before any
+// payload store.
+#include <cooperative_groups.h>
+
 #include "fqr_head.cuh"
 #include "fqr_launch.h"
 
@@ -434,64 +437,80 @@ __global__ void __launch_bounds__(kThreads) mla_quant_kernel(const MlaArgs a) {
   }
 }
 
-// Per-token scales: one block of up to 16 warps per row of Q at a time (each
-// warp's first two quads of heads held in registers), the row's maximum
-// reduced over the block before any payload store; the latent rows are warp
-// tasks first.
-constexpr int kTokenWarps = 16;
+// Per-token scales: a thread-block cluster of kTokenCluster blocks per row of
+// Q at a time.  The row's quads are spread over the cluster's warps (block r
+// takes quads r * nw + warp, then + kTokenCluster * nw, ...; each warp keeps
+// its first quad in registers and reads any further ones again for the
+// payloads).  The row's maximum is reduced over each warp (shuffles), each
+// block (shared memory) and the cluster: every block reads its peers'
+// partial maxima from their shared memory (distributed shared memory, after
+// a cluster barrier), so no global memory and no second kernel is involved.
+// The latent rows are warp tasks spread over the clusters.
+constexpr int kTokenWarps = 16;   // warps per block at most
+constexpr int kTokenCluster = 4;  // blocks per cluster (one row of Q)
 
 template <int FP8, int STYLE>
 __global__ void __launch_bounds__(kTokenWarps * 32) mla_token_kernel(const MlaArgs a) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ int smem[];
   int* s_indptr = smem;
   int* s_seq = s_indptr + a.B + 1;
-  float* s_red = reinterpret_cast<float*>(s_seq + a.B);  // one float per warp
+  float* s_red = reinterpret_cast<float*>(s_seq + a.B);  // one float per warp, then the block's
   const int lane = threadIdx.x & 31;
   const int warp = __shfl_sync(0xffffffffu, static_cast<int>(threadIdx.x >> 5), 0);
   const int nw = blockDim.x >> 5;
   const int g = lane >> 3, l8 = lane & 7;
-  const int gwarp = blockIdx.x * nw + warp;
+  const int crank = static_cast<int>(cluster.block_rank());
+  const int cid = blockIdx.x / kTokenCluster;       // this block's cluster
+  const int ncl = gridDim.x / kTokenCluster;        // clusters in the grid
+  const int cw = crank * nw + warp;                 // warp index inside the cluster
+  const int cwarps = kTokenCluster * nw;
+  // latent rows: warp task pw, pw + (all warps), ... with the warps ordered
+  // cluster-minor, so that consecutive rows go to different clusters
+  const int pw = cw * ncl + cid;
   const int nwarps = gridDim.x * nw;
 
-  // before the wait: metadata, this warp's latent row and the block's first
-  // row of Q into L2 (see mla_prefetch)
-  mla_prefetch(a, gwarp < a.T ? gwarp : INT64_MAX, lane);
-  if (blockIdx.x < a.T) {
-    const uint16_t* qrow = a.q + static_cast<int64_t>(blockIdx.x) * a.q_tok;
-    const int64_t lines = (static_cast<int64_t>(a.Hq) * a.q_head + 63) / 64;
-    for (int64_t l = threadIdx.x; l < lines; l += blockDim.x) prefetch_l2(qrow + 64 * l);
+  // before the wait: metadata, this warp's first latent row and this block's
+  // quads of the cluster's first row of Q into L2 (see mla_prefetch)
+  mla_prefetch(a, pw < a.T ? pw : INT64_MAX, lane);
+  if (cid < a.T) {
+    const uint16_t* qrow = a.q + static_cast<int64_t>(cid) * a.q_tok;
+    const int h = (crank * nw + warp) * 4 + lane;
+    if (lane < 4 && h < a.Hq) {
+      const uint16_t* hp = qrow + static_cast<int64_t>(h) * a.q_head;
+      for (int e = 0; e < a.nope + kRope; e += 64) prefetch_l2(hp + e);
+    }
   }
   grid_dependency_wait();
   grid_launch_dependents();
   const Meta m{a.q_indptr, a.seq_lens, a.positions, a.flags, a.T, a.B,
                static_cast<int64_t>(a.max_blocks) * a.block_size, a.cs_rows};
+  // (every block of every cluster reaches the same verdict: a malformed batch
+  // returns them all before any cluster barrier)
   if (stage_and_validate(m, s_indptr, s_seq)) return;
 
-  for (int t = gwarp; t < a.T; t += nwarps) {  // latent rows
+  for (int t = pw; t < a.T; t += nwarps) {  // latent rows
     const int b = request_of_row(s_indptr, a.B, t);
     const int p_slot = t + s_seq[b] - s_indptr[b + 1];
     const int64_t pos = a.positions != nullptr ? a.positions[t] : static_cast<int64_t>(p_slot);
     latent_row<FP8, STYLE>(a, t, b, p_slot, a.cs + pos * kRope, lane);
   }
   const int W = a.nope + kRope;
-  for (int t = blockIdx.x; t < a.T; t += gridDim.x) {  // Q rows (block-uniform loop)
+  for (int t = cid; t < a.T; t += ncl) {  // Q rows (cluster-uniform loop)
     const int b = request_of_row(s_indptr, a.B, t);
     const int p_slot = t + s_seq[b] - s_indptr[b + 1];
     const int64_t pos = a.positions != nullptr ? a.positions[t] : static_cast<int64_t>(p_slot);
     float c[4], s[4];
     mla_cos_sin<STYLE>(a.cs + pos * kRope, l8, c, s);
     const uint16_t* qrow = a.q + static_cast<int64_t>(t) * a.q_tok;
-    // pass 1: the row's maximum.  The warp's first two quads are loaded
-    // together and stay in registers; any further quads are read again.
-    const int hA = warp * 4 + g, hB = hA + 4 * nw;
-    const bool okA = hA < a.Hq, okB = hB < a.Hq;  // (group-uniform)
-    QHead va, vb;
+    // pass 1: the maximum over this warp's quads
+    const int hA = cw * 4 + g;
+    const bool okA = hA < a.Hq;  // (group-uniform)
+    QHead va;
     if (okA) load_q_head<STYLE>(qrow + static_cast<int64_t>(hA) * a.q_head, a.nope, l8, c, s, va);
-    if (okB) load_q_head<STYLE>(qrow + static_cast<int64_t>(hB) * a.q_head, a.nope, l8, c, s, vb);
-    float mx = 0.0f;
-    if (okA) mx = q_head_amax(va, a.nope, l8);
-    if (okB) mx = fmaxf(mx, q_head_amax(vb, a.nope, l8));
-    for (int h = hA + 8 * nw; h - g < a.Hq; h += 4 * nw) {
+    float mx = okA ? q_head_amax(va, a.nope, l8) : 0.0f;
+    for (int h = hA + 4 * cwarps; h - g < a.Hq; h += 4 * cwarps) {
       if (h < a.Hq) {
         QHead v;
         load_q_head<STYLE>(qrow + static_cast<int64_t>(h) * a.q_head, a.nope, l8, c, s, v);
@@ -502,23 +521,29 @@ __global__ void __launch_bounds__(kTokenWarps * 32) mla_token_kernel(const MlaAr
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if (lane == 0) s_red[warp] = mx;
     __syncthreads();
-    mx = s_red[0];
-    for (int i = 1; i < nw; ++i) mx = fmaxf(mx, s_red[i]);
+    if (threadIdx.x == 0) {
+      float bm = s_red[0];
+      for (int i = 1; i < nw; ++i) bm = fmaxf(bm, s_red[i]);
+      s_red[nw] = bm;
+    }
+    cluster.sync();  // every block's partial maximum is in its shared memory
+    mx = 0.0f;
+#pragma unroll
+    for (int r = 0; r < kTokenCluster; ++r) mx = fmaxf(mx, *cluster.map_shared_rank(s_red + nw, r));
+    cluster.sync();  // read everywhere before any block reuses s_red or exits
     const float sc = __fdiv_rn(fmaxf(mx, 1e-6f), a.upper_max);
     const float rc = __frcp_rn(sc);
-    if (threadIdx.x == 0) a.q_scale[t] = sc;
+    if (crank == 0 && threadIdx.x == 0) a.q_scale[t] = sc;
     // pass 2: payloads
     unsigned char* orow = a.q_out + static_cast<int64_t>(t) * a.Hq * W;
     if (okA) store_q_head<FQR_MLA_Q_TOKEN>(va, orow + static_cast<int64_t>(hA) * W, a.nope, l8, 0.0f, sc, rc);
-    if (okB) store_q_head<FQR_MLA_Q_TOKEN>(vb, orow + static_cast<int64_t>(hB) * W, a.nope, l8, 0.0f, sc, rc);
-    for (int h = hA + 8 * nw; h - g < a.Hq; h += 4 * nw) {
+    for (int h = hA + 4 * cwarps; h - g < a.Hq; h += 4 * cwarps) {
       if (h < a.Hq) {
         QHead v;
         load_q_head<STYLE>(qrow + static_cast<int64_t>(h) * a.q_head, a.nope, l8, c, s, v);
         store_q_head<FQR_MLA_Q_TOKEN>(v, orow + static_cast<int64_t>(h) * W, a.nope, l8, 0.0f, sc, rc);
       }
     }
-    __syncthreads();  // s_red is reused by the block's next row
   }
 }
 
@@ -550,17 +575,21 @@ int launch_mla(const fqr_mla_params& p, cudaStream_t stream) {
   if (p.q_quant == FQR_MLA_Q_TOKEN) {
     MlaKernel k = p.cache_fp8 ? (p.rope_style == 0 ? mla_token_kernel<1, 0> : mla_token_kernel<1, 1>)
                               : (p.rope_style == 0 ? mla_token_kernel<0, 0> : mla_token_kernel<0, 1>);
-    const int nw = a.qgroups < kTokenWarps ? a.qgroups : kTokenWarps;  // warps per block
-    const size_t smem = static_cast<size_t>(2 * p.B + 1) * sizeof(int) + nw * sizeof(float);
+    // warps per block: the row's quads spread over the cluster, one per warp
+    // while they last (at most kTokenWarps)
+    const int per_block = (a.qgroups + kTokenCluster - 1) / kTokenCluster;
+    const int nw = per_block < kTokenWarps ? (per_block > 0 ? per_block : 1) : kTokenWarps;
+    const size_t smem = static_cast<size_t>(2 * p.B + 1) * sizeof(int) + (nw + 1) * sizeof(float);
     DeviceInfo d;
     int per_sm = 0;
     if (device_info(&d) != FQR_OK ||
         resident_blocks(reinterpret_cast<const void*>(k), 32 * nw, smem, &per_sm) != FQR_OK)
       return FQR_ECUDA;
-    const int sms = d.sms;
-    const int64_t cap = static_cast<int64_t>(per_sm) * sms;
+    // clusters: one per row, at most as many as fit on the device at once
+    const int64_t cap = static_cast<int64_t>(per_sm) * d.sms / kTokenCluster;
     const int64_t want = p.T > 0 ? p.T : 1;
-    return launch_pdl(k, static_cast<int>(want < cap ? want : cap), 32 * nw, smem, stream, a);
+    const int clusters = static_cast<int>(want < cap ? want : (cap > 0 ? cap : 1));
+    return launch_pdl(k, clusters * kTokenCluster, 32 * nw, smem, stream, a, kTokenCluster);
   }
   if (p.q_quant != FQR_MLA_Q_NONE) {
     MlaKernel k = p.q_quant == FQR_MLA_Q_STATIC ? select_quant<FQR_MLA_Q_STATIC>(p.cache_fp8, p.rope_style)

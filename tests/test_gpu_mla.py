@@ -96,6 +96,24 @@ def test_mla_q_fp8_ragged(q_quant, style, upper):
     run(w)
 
 
+@pytest.mark.parametrize("style", [1, 0])
+def test_mla_q_fp8_per_token_wide_rows_many_clusters(style):
+    """Per-token scales with 288 heads (72 quads: the cluster's 64 warps take
+    a second quad each for 8 of them) and 50 rows of 1-2 tokens per request
+    (more rows than the device holds clusters of one row each)."""
+    rng = np.random.default_rng(40 + style)
+    B = 30
+    n = rng.integers(1, 3, B)
+    L = rng.integers(2, 300, B) + n
+    w = workloads.make_mla(seed=41 + style, n_new=n, seq_lens=L, Hq=288, block_size=64,
+                           max_blocks=int(np.ceil(L.max() / 64)) + 1, rope_style=style,
+                           kv_lora_rank=512, cos_sin_rows=int(L.max()) + 1, q_quant=2,
+                           upper_max=448.0)
+    assert w.T >= 40
+    w.q[3] = 0                                  # an all-zero token (floor scale)
+    run(w)
+
+
 @pytest.mark.parametrize("q_quant", [1, 2, 3])
 def test_mla_q_fp8_malformed_writes_nothing(q_quant):
     w = workloads.make_mla(seed=4, n_new=[2, 1, 1], seq_lens=[4, 3, 2], Hq=8, block_size=4,
