@@ -71,6 +71,8 @@ def parse_args(argv=None):
                     help="profiling run: only --workload (or mla_decode), --steps eager launches, "
                          "no graphs, no e2e / per-config / CPU legs, no JSON line")
     ap.add_argument("--mla", action="store_true", help="with --profile: the MLA workload")
+    ap.add_argument("--mla-workload", default="mla_decode", choices=sorted(workloads.MLA_CONFIGS),
+                    help="with --profile --mla: which MLA workload")
     ap.add_argument("--small-cache", action="store_true",
                     help="with --profile: wrap sequence lengths to 1024 (same bytes per call, "
                          "a cache of 1024 slots per request)")
@@ -691,7 +693,7 @@ def main(argv=None):
 def run_profile(args, torch, fqr, dev):
     """A few eager launches of one workload for ncu (small device footprint)."""
     if args.mla:
-        b = MlaBench(torch, fqr, dev, max_replicas=args.replicas or 2)
+        b = MlaBench(torch, fqr, dev, max_replicas=args.replicas or 2, name=args.mla_workload)
     else:
         b = AppendBench(args.workload, torch, fqr, dev, max_replicas=args.replicas or 2,
                         schedule=args.schedule, small_cache=args.small_cache)

@@ -4,10 +4,11 @@
 // Method: FlashInfer PR #5956, section "Contract" (see fqr_head.cuh for the
 // per-head arithmetic).
 //
-//   * head task = 4 heads of one packed row (8 lanes per head); the task's two
-//     16-byte loads per lane need no metadata and are issued before the
-//     validation prologue; the next task's loads are issued before the current
-//     task is computed.
+//   * head task = 4 heads of one packed row (8 lanes per head), in quad-major
+//     order (consecutive warps take the same quad of consecutive rows); the
+//     task's two 16-byte loads per lane need no metadata and are issued before
+//     the validation prologue; the next task's loads are issued before the
+//     current task is computed.
 //   * the first task also reads its own request's metadata in that first
 //     round trip (request guessed as b = t) and, when it is consistent and
 //     in bounds, issues its page-id and cos/sin loads before the prologue, so
@@ -31,9 +32,8 @@ namespace fqr {
 
 struct WarpArgs {
   HeadParams hp;
-  FastDiv qdiv;  // division by quads
-  FastDiv tdiv;  // division by T (quad-major order)
-  int quad_major;  // head task order: quad-major (w = quad * T + t) or row-major
+  FastDiv qdiv;  // division by quads (tail shares)
+  FastDiv tdiv;  // division by T (head task -> quad, row)
   const uint16_t* qkv;
   int64_t row_stride;
   int T, B, H, quads, n_head;
@@ -59,19 +59,17 @@ __host__ __device__ __forceinline__ int warp_zero_offset(int B) {
   return ((2 * kHeadDim + 2 * B + 1) * static_cast<int>(sizeof(int)) + 15) & ~15;
 }
 
-// Packed row t and quad of head task w.  Row-major order keeps a row's quads
-// on consecutive warps; quad-major order gives consecutive warps the same
-// quad of consecutive rows, so a block's warps serve different requests and
-// share their tails (one share per quad) -- an SM then zeroes parts of many
-// requests' tails instead of all of one.
+// Packed row t and quad of head task w, in quad-major order (w = quad * T +
+// t): consecutive warps take the same quad of consecutive rows, so a block's
+// warps serve different requests and each writes one share of its request's
+// tail -- an SM zeroes parts of many requests' tails, not all of one.
+// (Measured on B200 against row-major order, which put a row's quads on
+// consecutive warps: Qwen3-style decode 3.51 -> 3.20 us per launch, FP8
+// decode with 256 rows 8.58 -> 8.28 us, tiny decode 2.49 -> 2.25 us; there
+// the SMs with the largest tails set the launch time.)
 __device__ __forceinline__ void head_task(const WarpArgs& a, int w, int& t, int& quad) {
-  if (a.quad_major) {
-    quad = static_cast<int>(a.tdiv.div(static_cast<uint32_t>(w)));
-    t = w - quad * a.T;
-  } else {
-    t = static_cast<int>(a.qdiv.div(static_cast<uint32_t>(w)));
-    quad = w - t * a.quads;
-  }
+  quad = static_cast<int>(a.tdiv.div(static_cast<uint32_t>(w)));
+  t = w - quad * a.T;
 }
 
 __device__ __forceinline__ void warp_load_head(const WarpArgs& a, int w, int g, int l8, uint4& xa,
@@ -428,12 +426,6 @@ int launch_append_warp(const fqr_append_params& p, const HeadParams& hp, cudaStr
   a.n_head = static_cast<int>(n_head);
   a.qdiv = FastDiv(static_cast<uint32_t>(a.quads));
   a.tdiv = FastDiv(static_cast<uint32_t>(p.T > 0 ? p.T : 1));
-  // Quad-major task order: measured on B200 against row-major, Qwen3-style
-  // decode 3.51 -> 3.20 us per launch, FP8 decode (256 rows) 8.58 -> 8.28 us,
-  // tiny decode 2.49 -> 2.25 us; with row-major order a block held one row,
-  // so one SM zeroed one request's whole tail and the SMs with the largest
-  // tails set the launch time.
-  a.quad_major = 1;
   a.qw = p.q_norm_w;
   a.kw = p.k_norm_w;
   a.cs = p.cos_sin_cache;
