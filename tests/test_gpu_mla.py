@@ -115,6 +115,32 @@ def test_mla_q_fp8_per_token_wide_rows_many_clusters(style):
 
 
 @pytest.mark.parametrize("q_quant", [1, 2, 3])
+def test_mla_q_fp8_with_bf16_latent(q_quant):
+    """FP8 Q with a BF16 latent cache (every kernel variant's FP8 = 0 side)."""
+    rng = np.random.default_rng(60 + q_quant)
+    n = rng.integers(1, 4, 6)
+    L = rng.integers(1, 90, 6) + n
+    w = workloads.make_mla(seed=61 + q_quant, n_new=n, seq_lens=L, Hq=20, block_size=32,
+                           max_blocks=int(np.ceil(L.max() / 32)) + 1, kv_lora_rank=128,
+                           cos_sin_rows=int(L.max()) + 1, cache_fp8=0, q_quant=q_quant,
+                           q_scale_inv=25.0)
+    run(w)
+
+
+@pytest.mark.parametrize("Hq", [4, 8, 20])
+def test_mla_q_fp8_per_token_few_heads(Hq):
+    """Per-token scales with fewer quads than the cluster has blocks: the
+    blocks without a quad still take part in the cluster's maximum."""
+    rng = np.random.default_rng(70 + Hq)
+    n = rng.integers(1, 3, 5)
+    L = rng.integers(1, 60, 5) + n
+    w = workloads.make_mla(seed=71 + Hq, n_new=n, seq_lens=L, Hq=Hq, block_size=16,
+                           max_blocks=int(np.ceil(L.max() / 16)) + 1, kv_lora_rank=64,
+                           cos_sin_rows=int(L.max()) + 1, q_quant=2)
+    run(w)
+
+
+@pytest.mark.parametrize("q_quant", [1, 2, 3])
 def test_mla_q_fp8_malformed_writes_nothing(q_quant):
     w = workloads.make_mla(seed=4, n_new=[2, 1, 1], seq_lens=[4, 3, 2], Hq=8, block_size=4,
                            max_blocks=2, kv_lora_rank=64, cos_sin_rows=8, q_quant=q_quant)
