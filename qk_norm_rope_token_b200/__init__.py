@@ -6,7 +6,9 @@ fails if the library has not been built (python
 qk_norm_rope_token_b200/build.py).
 
     append_paged(...)       -> fqr_append_paged
+    append_plan(params)     -> fqr_append_plan_query (the launch, without launching)
     concat_mla_cache(...)   -> fqr_concat_mla_cache
+    StagedAppend            -> fqr_pipeline_* (pinned-host batches, pipelined)
 
 Tensors: BF16 data as torch.bfloat16 (or int16/uint16 bit patterns), FP8 E4M3
 as torch.float8_e4m3fn or torch.uint8.  All on one CUDA device.

@@ -69,3 +69,21 @@ def test_reference_arm_rank0_prints_one_line(capsys):
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["value"] > 0 and rec["unit"] == "tokens/s"
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_describe_plan_names_the_schedule_and_variants():
+    """The bench's `kernel` field is the launch fqr_append_plan_query reports,
+    in words (checked here on plans shaped like the library's)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    lat = dict(schedule=1, grid=139, block_threads=384, tasks=1664, warp_check=1, bulk_tails=0,
+               request_tails=0)
+    d = bench.describe_plan(lat)
+    assert "latency schedule" in d and "139 blocks of 384 threads" in d
+    assert "1664 warp tasks" in d and "warp-level batch check" in d and "bulk" not in d
+    d = bench.describe_plan(dict(lat, warp_check=0, bulk_tails=1, request_tails=1))
+    assert "block batch prologue" in d and "bulk-copy tails" in d and "own the tails" in d
+    d = bench.describe_plan(dict(schedule=2, grid=296, block_threads=288, tasks=9212,
+                                 warp_check=0, bulk_tails=0, request_tails=0))
+    assert "streaming schedule" in d and "296 blocks of 288 threads" in d and "9212 units" in d
