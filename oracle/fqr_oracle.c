@@ -105,14 +105,25 @@ void fqro_f32_to_bf16_array(const float* x, uint16_t* out, int64_t n) {
 
 /* RMSNorm over one head ([TRT] review excerpt; [FI] "per-head RMSNorm eps
  * 1e-6"): mean square over all n elements, eps inside the square root, then
- * scale and weight.  Sequential fp32 sum of rounded squares. */
+ * scale and weight.
+ *
+ * The mean square is the fp32 rounding of the exact mean of the squares
+ * ([FI] "What changes": an fp32 reference of the norm; the sum itself has no
+ * stated order, so no order is taken).  The squares are formed and summed in
+ * binary64: a BF16 value has 8 significant bits, so its square has 16, and
+ * the binary64 sum of 128 of them is exact whenever the head's nonzero
+ * magnitudes span at most 2^15 (2 * 15 + 16 + 7 <= 53 bits); beyond that it
+ * is within 2^-46 of the exact sum, far inside one fp32 rounding.  The sum is
+ * then divided by n and rounded once to fp32; eps is added, and the square
+ * root and the reciprocal are taken, each as one correctly rounded fp32
+ * operation. */
 void fqro_rmsnorm(const float* x, const float* w, int n, float eps, float* y) {
-  float ss = 0.0f;
+  double ss = 0.0;
   for (int i = 0; i < n; ++i) {
-    float sq = x[i] * x[i];
+    double sq = (double)x[i] * (double)x[i];
     ss = ss + sq;
   }
-  float ms = ss / (float)n;
+  float ms = (float)(ss / (double)n);
   float inv = 1.0f / sqrtf(ms + eps);
   for (int i = 0; i < n; ++i) {
     float t = x[i] * inv;

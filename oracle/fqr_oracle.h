@@ -38,7 +38,8 @@ void fqro_f32_to_e4m3_array(const float* x, uint8_t* out, int64_t n);
 void fqro_f32_to_bf16_array(const float* x, uint16_t* out, int64_t n);
 
 /* ---- per-head steps ----------------------------------------------------- */
-/* y = x * (1 / sqrt(sum(x^2)/n + eps)) * w   (w == NULL -> w = 1) */
+/* y = x * (1 / sqrt(sum(x^2)/n + eps)) * w   (w == NULL -> w = 1); the mean
+ * square is the fp32 rounding of the binary64 mean of the squares */
 void fqro_rmsnorm(const float* x, const float* w, int n, float eps, float* y);
 /* NeoX rotate-half on y[0, rot): pairs (i, i + rot/2) with cs = [cos | sin] */
 void fqro_rope_neox(float* y, const float* cs_row, int rot);

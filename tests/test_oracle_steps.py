@@ -1,5 +1,7 @@
 """Pins of the oracle's per-head steps (RMSNorm, NeoX and GPT-J RoPE) against
 closed forms, invariants and complex multiplication."""
+from fractions import Fraction
+
 import numpy as np
 import pytest
 
@@ -55,6 +57,74 @@ def test_rmsnorm_scale_relation(c):
     msc = np.mean(xc.astype(np.float64) ** 2)
     ratio = np.sqrt((ms + eps) / (msc + eps)) * (msc / ms) ** 0.5
     assert np.allclose(y2, y1 * ratio, rtol=2e-6, atol=1e-30)
+
+
+def _bf16_valued(a):
+    """float32 values truncated to BF16 (8 significant bits), as the packed
+    rows deliver them."""
+    a = np.asarray(a, np.float32)
+    return (a.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+
+
+def _round_to_f32(q: Fraction) -> np.float32:
+    """Round an exact rational to the nearest binary32 (ties to even), from
+    the definition: the quantum of q's binade, an integer count of quanta
+    rounded half-to-even, and the result rebuilt (normal range only)."""
+    if q == 0:
+        return np.float32(0.0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    quantum = Fraction(2) ** (e - 23)
+    n, rem = divmod(a, quantum)
+    if rem * 2 > quantum or (rem * 2 == quantum and n % 2 == 1):
+        n += 1
+    return np.float32(sign * float(n * quantum))
+
+
+@pytest.mark.parametrize("scale", [1e-3, 1.0, 40.0])
+def test_rmsnorm_sum_is_order_free(scale):
+    """The mean square is a function of the multiset of squares: permuting a
+    head's elements permutes its output, bit for bit.  A sequential fp32 sum
+    depends on the order and fails this on some of these heads."""
+    for _ in range(60):
+        x = _bf16_valued(rng.standard_normal(D) * scale)
+        y = oracle.rmsnorm(x, None, 1e-6)
+        for _ in range(4):
+            p = rng.permutation(D)
+            assert np.array_equal(oracle.rmsnorm(x[p], None, 1e-6), y[p])
+
+
+def test_rmsnorm_mean_square_is_the_rounded_exact_mean():
+    """y = x * (1 / sqrt(ms + eps)) with ms the binary32 rounding of the exact
+    rational mean of the squares (computed here with exact fractions), then
+    IEEE fp32 addition, square root and reciprocal."""
+    eps = np.float32(1e-6)
+    for scale in (1e-2, 0.7, 3.0, 250.0):
+        for _ in range(25):
+            x = _bf16_valued(rng.standard_normal(D) * scale)
+            s = sum(Fraction(float(v)) ** 2 for v in x)
+            ms = _round_to_f32(s / D)
+            inv = np.float32(1.0) / np.sqrt(np.float32(ms + eps))
+            want = (x * inv).astype(np.float32)
+            assert np.array_equal(oracle.rmsnorm(x, None, float(eps)), want)
+
+
+def test_rmsnorm_large_element_beside_small_ones():
+    """x = (4096, 1, ..., 1): the squares sum to 2^24 + 127 exactly, which a
+    running fp32 sum rounds away to 2^24 (every +1 is lost), shifting y_0 by
+    about 3.8e-6 relative.  The closed form of the exact mean square is
+    y_0 = 4096 / sqrt((2^24 + 127) / 128 + eps)."""
+    x = np.ones(D, np.float32)
+    x[0] = 4096.0
+    y = oracle.rmsnorm(x, None, 1e-6).astype(np.float64)
+    ms = (2.0 ** 24 + 127) / 128
+    assert y[0] == pytest.approx(4096 / np.sqrt(ms + 1e-6), rel=2.5e-7)
+    assert y[1] == pytest.approx(1 / np.sqrt(ms + 1e-6), rel=2.5e-7)
 
 
 def test_rmsnorm_weight_applies_after_normalisation():
