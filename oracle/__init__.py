@@ -54,7 +54,7 @@ class _MlaArgs(ctypes.Structure):
         ("latent_cache", c_vp), ("num_blocks", c_i32), ("block_size", c_i32),
         ("cache_fp8", c_i32), ("kv_scale", c_f32), ("flags", c_vp),
         ("q_quant", c_i32), ("q_scale_inv", c_f32), ("upper_max", c_f32),
-        ("q_out", c_vp), ("q_scale", c_vp),
+        ("q_out", c_vp), ("q_scale", c_vp), ("q_group", c_i32),
     ]
 
 
@@ -204,7 +204,7 @@ def new_mla_q_outputs(w):
     """q_out [T, Hq, nope + rope] and q_scale ([T] per token, [T, Hq] per
     head) of the MLA Q quantisation, pre-filled with sentinels."""
     q_out = np.full((w.T, w.Hq, w.nope_dim + w.rope_dim), 0xFF, np.uint8)
-    shape = {2: (w.T,), 3: (w.T, w.Hq)}.get(w.q_quant, (1,))
+    shape = w.q_scale_shape
     return q_out, np.full(shape, np.nan, np.float32)
 
 
@@ -237,7 +237,8 @@ def concat_mla_cache(w, q: np.ndarray, latent: np.ndarray, flags: np.ndarray, *,
         latent_cache=_ptr(latent), num_blocks=latent.shape[0],
         block_size=w.block_size, cache_fp8=w.cache_fp8, kv_scale=w.kv_scale,
         flags=_ptr(flags), q_quant=w.q_quant, q_scale_inv=w.q_scale_inv,
-        upper_max=w.upper_max, q_out=_ptr(q_out), q_scale=_ptr(q_scale))
+        upper_max=w.upper_max, q_out=_ptr(q_out), q_scale=_ptr(q_scale),
+        q_group=w.q_group)
     return lib().fqro_concat_mla_cache(ctypes.byref(a))
 
 

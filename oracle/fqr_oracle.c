@@ -341,6 +341,22 @@ static void quantize_q(const fqro_mla_args* a, int64_t r, const float* cs) {
   const int W = a->nope_dim + a->rope_dim;
   float v[1024];
   float s = 0.0f;
+  if (a->q_quant == 4) {  /* one scale per group of q_group values of a head */
+    const int G = a->q_group, ng = (W + G - 1) / G;
+    for (int h = 0; h < a->Hq; ++h) {
+      mla_q_values(a, r, h, cs, v);
+      uint8_t* out = a->q_out + (r * a->Hq + h) * W;
+      for (int k = 0; k < ng; ++k) {
+        const int lo = k * G, hi = lo + G < W ? lo + G : W;
+        float amax = 0.0f;
+        for (int i = lo; i < hi; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        s = fmaxf(amax, 1e-6f) / a->upper_max;
+        a->q_scale[(r * a->Hq + h) * ng + k] = s;
+        for (int i = lo; i < hi; ++i) out[i] = fqro_f32_to_e4m3_rn_satfinite(v[i] / s);
+      }
+    }
+    return;
+  }
   if (a->q_quant == 2) {  /* one scale for the whole token */
     float amax = 0.0f;
     for (int h = 0; h < a->Hq; ++h) {
@@ -373,6 +389,7 @@ int fqro_concat_mla_cache(const fqro_mla_args* a) {
   const int R = a->rope_dim, K = a->kv_lora_rank, W = K + R;
   float y[512];
   if (R > 512 || a->nope_dim + R > 1024) return 2;
+  if (a->q_quant == 4 && a->q_group < 1) return 2;
   for (int32_t b = 0; b < a->B; ++b) {
     int64_t lo = a->q_indptr[b], hi = a->q_indptr[b + 1], L = a->seq_lens[b];
     for (int64_t r = lo; r < hi; ++r) {

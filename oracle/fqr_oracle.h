@@ -121,11 +121,15 @@ typedef struct {
    *   1 static per-tensor:     e4m3(v * q_scale_inv)
    *   2 dynamic per-token:     s = max(max |v| over the token, 1e-6) / upper_max,
    *                            e4m3(v / s), q_scale [T]
-   *   3 dynamic per-head:      the same with the max over one head, q_scale [T, Hq] */
+   *   3 dynamic per-head:      the same with the max over one head, q_scale [T, Hq]
+   *   4 dynamic per-group:     the same with the max over each group of q_group
+   *                            consecutive values of a head (the last group of a
+   *                            head may be shorter), q_scale [T, Hq, ceil(W / q_group)] */
   int32_t q_quant;
   float q_scale_inv, upper_max;
   uint8_t* q_out;
   float* q_scale;
+  int32_t q_group;            /* elements per group (q_quant 4), >= 1          */
 } fqro_mla_args;
 
 int fqro_concat_mla_cache(const fqro_mla_args* a);

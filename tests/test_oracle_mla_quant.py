@@ -117,3 +117,74 @@ def test_flagged_call_writes_no_q_output():
     rc, *_ = run(w, q_out=q_out, q_scale=q_scale, q_indptr=np.array([0, 2, 1, 6], np.int32))
     assert rc == 1
     assert np.array_equal(q_out, q0) and np.array_equal(q_scale, s0, equal_nan=True)
+
+
+# ---------------------------------------------------------- per-group scales
+
+def small_group(G, seed=3, upper=448.0):
+    w = small(4, seed=seed, upper=upper)
+    w.q_group = G
+    return w
+
+
+@pytest.mark.parametrize("upper", [448.0, 240.0])
+@pytest.mark.parametrize("G", [8, 64, 128, 192])
+def test_group_scale_invariants(G, upper):
+    """Each group of G consecutive values of a head (the last one shorter when
+    G does not divide the head width) has s = max|v| / upper_max, holds a code
+    of exactly +-upper_max at its maximum, and dequantises within E4M3
+    precision."""
+    w = small_group(G, upper=upper)
+    rc, _, _, _, q_out, q_scale = run_q(w)
+    assert rc == 0
+    W = w.nope_dim + w.rope_dim
+    ng = -(-W // G)
+    assert q_scale.shape == (w.T, w.Hq, ng)
+    top = e4m3_brute(np.float32(upper))
+    for r in range(w.T):
+        v = values(w, r)
+        dec = e4m3_decode(q_out[r])
+        for h in range(w.Hq):
+            for k in range(ng):
+                sl = slice(k * G, min(W, (k + 1) * G))
+                s = float(q_scale[r, h, k])
+                assert s == pytest.approx(np.abs(v[h, sl]).max() / upper, rel=1e-6)
+                assert np.abs(dec[h, sl]).max() == upper
+                assert ((q_out[r, h, sl] & 0x7F) == top).any()
+                err = np.abs(dec[h, sl] * s - v[h, sl])
+                assert np.all(err <= np.abs(v[h, sl]) * 2.0 ** -4 + s * 2.0 ** -10 + 1e-30)
+
+
+@pytest.mark.parametrize("G", [192, 256, 1000])
+def test_group_as_wide_as_the_head_is_the_per_head_scale(G):
+    """G >= nope + rope: one group per head, bit for bit the per-head mode."""
+    wg, wh = small_group(G), small(3)
+    _, _, _, _, qg, sg = run_q(wg)
+    _, _, _, _, qh, sh = run_q(wh)
+    assert np.array_equal(qg, qh)
+    assert np.array_equal(sg[..., 0], sh)
+
+
+def test_group_of_128_splits_nope_and_rope():
+    """With nope 128 and rope 64, G = 128 gives two groups per head: the nope
+    part (raw BF16 values) and the rotated rope part."""
+    w = small_group(128)
+    rc, _, _, _, q_out, q_scale = run_q(w)
+    for r in range(w.T):
+        v = values(w, r)
+        assert np.allclose(q_scale[r, :, 0], np.abs(v[:, :128]).max(axis=1) / w.upper_max,
+                           rtol=1e-6)
+        assert np.allclose(q_scale[r, :, 1], np.abs(v[:, 128:]).max(axis=1) / w.upper_max,
+                           rtol=1e-6)
+
+
+def test_all_zero_group():
+    """A group whose values are all zero gets the floor scale 1e-6 / upper_max
+    and zero codes; the head's other groups are unaffected."""
+    w = small_group(64)
+    w.q[1, 2, :64] = 0          # the first group of head 2 of row 1
+    rc, _, _, _, q_out, q_scale = run_q(w)
+    assert rc == 0
+    assert q_scale[1, 2, 0] == np.float32(1e-6) / np.float32(w.upper_max)
+    assert np.all(e4m3_decode(q_out[1, 2, :64]) == 0)
+    assert q_scale[1, 2, 1] > 1e-4 and np.abs(e4m3_decode(q_out[1, 2, 64:])).max() == w.upper_max

@@ -131,9 +131,17 @@ class MlaWorkload:
     block_size: int
     cache_fp8: int
     kv_scale: float
-    q_quant: int = 0           # 0 none, 1 static, 2 dynamic per token, 3 per head
+    q_quant: int = 0           # 0 none, 1 static, 2 dynamic per token, 3 per head, 4 per group
     q_scale_inv: float = 1.0
     upper_max: float = 448.0
+    q_group: int = 0           # q_quant 4: values per group of a head
+
+    @property
+    def q_scale_shape(self) -> tuple:
+        """[T] per token, [T, Hq] per head, [T, Hq, ceil(W / q_group)] per group."""
+        W = self.nope_dim + self.rope_dim
+        return {2: (self.T,), 3: (self.T, self.Hq),
+                4: (self.T, self.Hq, -(-W // max(1, self.q_group)))}.get(self.q_quant, (1,))
 
     @property
     def kv_lora_rank(self) -> int:
@@ -231,12 +239,16 @@ def fp8_decode_dynamic(seed=1003) -> AppendWorkload:
                        v_scale=0.05, upper_max=448.0)
 
 
-def ragged_prefill_fp8(seed=1004) -> AppendWorkload:
+def ragged_prefill_fp8(seed=1004, n_new=None) -> AppendWorkload:
     """Ragged prefill, static FP8: 16 requests with U[0, 2048] new tokens (two
-    forced empty) on U[0, 4096] prior context, page 16, Hq 64 / Hkv 8."""
+    forced empty) on U[0, 4096] prior context, page 16, Hq 64 / Hkv 8.
+    n_new: keep these per-request token counts instead of the drawn ones (a
+    batch of the same shape with other data, positions and pages)."""
     rng = rng_for(seed + 7)
     n = rng.integers(0, 2048, size=16, endpoint=True)
     n[rng.choice(16, size=2, replace=False)] = 0
+    if n_new is not None:
+        n = np.asarray(n_new, dtype=np.int64).copy()
     prior = rng.integers(0, 4096, size=16, endpoint=True)
     L = prior + n
     return make_append(name="ragged_prefill_fp8_B16_h64x8_p16", seed=seed,
@@ -257,12 +269,13 @@ def malformed_indptr(w: AppendWorkload, seed=1104) -> np.ndarray:
     return ind
 
 
-def mla_decode(seed=1005, q_quant=0) -> MlaWorkload:
+def mla_decode(seed=1005, q_quant=0, q_group=0) -> MlaWorkload:
     """MLA decode latent concat: 32 x 1 token, 128 query heads, q [32,128,192]
     with interleaved RoPE on dims 128..191 (theta 10000), kv_c [32, 512],
     k_pe [32, 64], FP8 latent cache [16384, 64, 576] with scale 0.02.
     q_quant > 0: the same call with Q quantised to FP8 E4M3 (1 static
-    per-tensor with q_scale_inv 1/0.02, 2 dynamic per token, 3 per head)."""
+    per-tensor with q_scale_inv 1/0.02, 2 dynamic per token, 3 per head,
+    4 per group of q_group values of a head)."""
     rng = rng_for(seed)
     B = T = 32
     Hq, nope, rope_dim, rank = 128, 128, 64, 512
@@ -275,21 +288,22 @@ def mla_decode(seed=1005, q_quant=0) -> MlaWorkload:
     perm = rng.permutation(num_blocks).astype(np.int32).reshape(B, max_blocks)
     cs = cos_sin_cache(32768, rope_dim, 10000.0)
     q_indptr = np.arange(B + 1, dtype=np.int32)
-    suffix = {0: "", 1: "_qfp8_static", 2: "_qfp8_token", 3: "_qfp8_head"}[q_quant]
+    suffix = {0: "", 1: "_qfp8_static", 2: "_qfp8_token", 3: "_qfp8_head",
+              4: f"_qfp8_group{q_group}"}[q_quant]
     return MlaWorkload(name="mla_decode_B32_h128_latent576_fp8" + suffix, seed=seed,
                        T=T, B=B, Hq=Hq, nope_dim=nope, rope_dim=rope_dim, q=q,
                        kv_c=kv_c, k_pe=k_pe, cos_sin=cs, rope_style=1,
                        positions=None, q_indptr=q_indptr, seq_lens=L,
                        block_table=perm.copy(), num_blocks=num_blocks,
                        block_size=block_size, cache_fp8=1, kv_scale=0.02,
-                       q_quant=q_quant, q_scale_inv=1 / 0.02)
+                       q_quant=q_quant, q_scale_inv=1 / 0.02, q_group=q_group)
 
 
 def make_mla(*, seed=0, n_new, seq_lens, Hq, block_size, max_blocks,
              num_blocks=None, nope_dim=128, rope_dim=64, kv_lora_rank=512,
              rope_style=1, theta=10000.0, cos_sin_rows=None, cache_fp8=1,
              kv_scale=0.02, positions=None, q_quant=0, q_scale_inv=1.0,
-             upper_max=448.0) -> MlaWorkload:
+             upper_max=448.0, q_group=0) -> MlaWorkload:
     rng = rng_for(seed)
     n_new = np.asarray(n_new, dtype=np.int64)
     seq_lens = np.asarray(seq_lens, dtype=np.int32)
@@ -315,7 +329,7 @@ def make_mla(*, seed=0, n_new, seq_lens, Hq, block_size, max_blocks,
                        seq_lens=seq_lens, block_table=table,
                        num_blocks=num_blocks, block_size=block_size,
                        cache_fp8=cache_fp8, kv_scale=kv_scale, q_quant=q_quant,
-                       q_scale_inv=q_scale_inv, upper_max=upper_max)
+                       q_scale_inv=q_scale_inv, upper_max=upper_max, q_group=q_group)
 
 
 def prefill_dynq_gemma(seed=1006, q_len=129) -> AppendWorkload:
@@ -367,7 +381,11 @@ APPEND_CONFIGS = {
 MLA_CONFIGS = {"mla_decode": mla_decode,
                "mla_decode_qfp8_static": lambda seed=1005: mla_decode(seed, q_quant=1),
                "mla_decode_qfp8_token": lambda seed=1005: mla_decode(seed, q_quant=2),
-               "mla_decode_qfp8_head": lambda seed=1005: mla_decode(seed, q_quant=3)}
+               "mla_decode_qfp8_head": lambda seed=1005: mla_decode(seed, q_quant=3),
+               "mla_decode_qfp8_group64": lambda seed=1005: mla_decode(seed, q_quant=4,
+                                                                       q_group=64),
+               "mla_decode_qfp8_group128": lambda seed=1005: mla_decode(seed, q_quant=4,
+                                                                        q_group=128)}
 
 
 # ---------------------------------------------------------------------------
@@ -420,7 +438,7 @@ def mla_bytes(w: MlaWorkload) -> dict:
     W = w.nope_dim + w.rope_dim
     if w.q_quant:   # the whole head read, quantised into q_out (one byte each)
         reads = T * w.Hq * W * 2
-        writes = T * w.Hq * W + {2: 4 * T, 3: 4 * T * w.Hq}.get(w.q_quant, 0)
+        writes = T * w.Hq * W + 4 * int(np.prod(w.q_scale_shape)) * (w.q_quant >= 2)
     else:           # the rope part rotated in place
         reads = T * w.Hq * w.rope_dim * 2
         writes = T * w.Hq * w.rope_dim * 2
