@@ -368,6 +368,30 @@ __device__ __forceinline__ int quad_kind(const HeadParams& a, int h0) {
   return kAnyHead;
 }
 
+// 1 / sqrt(mean(x^2) + eps) of the head whose lane slices (8 float2 pairs,
+// BF16 values) are y, over the 8-lane group gmask.  The mean square is the
+// fp32 rounding of the exact mean of the squares: a BF16 value has 8
+// significant bits, its square 16, and the binary64 sum of a head's 128
+// squares is exact whenever its nonzero magnitudes span at most 2^15 -- so no
+// summation order (four lane chains, then the group's xor tree) can change
+// it.  One rounding to fp32, then +eps, the square root and the reciprocal,
+// each correctly rounded.
+__device__ __forceinline__ float inv_rms(const float2* y, float eps, unsigned gmask) {
+  double s[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const double u = y[j].x, v = y[j].y;
+    s[(j & 1) * 2] = fma(u, u, s[(j & 1) * 2]);
+    s[(j & 1) * 2 + 1] = fma(v, v, s[(j & 1) * 2 + 1]);
+  }
+  double ss = (s[0] + s[1]) + (s[2] + s[3]);
+  ss += __shfl_xor_sync(gmask, ss, 4);
+  ss += __shfl_xor_sync(gmask, ss, 2);
+  ss += __shfl_xor_sync(gmask, ss, 1);
+  const float ms = __double2float_rn(ss * (1.0 / kHeadDim));
+  return __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
+}
+
 // Norm + RoPE + quantisation + store of head h of row r.  xa/xb: the lane's two
 // 16-byte slices of the packed head; cs_row: the row's fp32 [cos | sin]
 // (shared or global memory); wts: the norm weights (load_weights).  gmask:
@@ -403,17 +427,7 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
   const bool is_q = KIND == kQHead || (KIND == kAnyHead && h < a.Hq);
   // -------------------------------------------------------------- RMSNorm
   if (is_q ? a.has_qw : a.has_kw) {
-    float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc = fma2(y[j], y[j], acc);
-    float ss = acc.x + acc.y;
-    ss += __shfl_xor_sync(gmask, ss, 4);
-    ss += __shfl_xor_sync(gmask, ss, 2);
-    ss += __shfl_xor_sync(gmask, ss, 1);
-    // rsqrtf: at most 2 ulp from 1/sqrt (CUDA's documented bound), against
-    // the correctly rounded sqrt then reciprocal of the step-wise definition;
-    // the parity bar propagates the difference with that of the summation order
-    const float inv = rsqrtf(__fadd_rn(ss * (1.0f / kHeadDim), a.eps));
+    const float inv = inv_rms(y, a.eps, gmask);
     const float2 iv = make_float2(inv, inv);
     float2 w[8];
     load_weights(wts, is_q, l8, w);
@@ -424,12 +438,7 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
   // ----------------------------------------------------------------- RoPE
   if (STYLE == 0) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 ac = mul2(y[j], c[j]), bs = mul2(y[4 + j], s[j]);
-      const float2 bc = mul2(y[4 + j], c[j]), as = mul2(y[j], s[j]);
-      y[j] = add2(ac, make_float2(-bs.x, -bs.y));
-      y[4 + j] = add2(bc, as);
-    }
+    for (int j = 0; j < 4; ++j) rotate_pairs2(y[j], y[4 + j], c[j], s[j]);
   } else {  // dims >= rot_dim pass through untouched
     const int half = a.rot >> 1;
 #pragma unroll

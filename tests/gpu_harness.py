@@ -9,18 +9,19 @@ be byte-identical to its pre-call content.
 
 Bars (from the method's tolerance statement): bitwise for slots, flags,
 untouched bytes, zero tails and V copies; <= 1 BF16 ulp for BF16 results;
-<= 1 E4M3 ulp for FP8 payloads; q_scale relative error <= 1e-5.
+<= 1 E4M3 ulp for FP8 payloads; q_scale relative error <= 1e-5.  check()
+asserts these on every element and reports the fraction of payloads and
+scales that are bit-identical; tests that expect bit-identical results (both
+sides evaluate the same correctly rounded steps) assert that on the report.
 """
 from __future__ import annotations
-
-import math
 
 import numpy as np
 import torch
 
 import oracle
 import qk_norm_rope_token_b200 as fqr
-from tests._util import bf16_bits_to_f32, e4m3_decode, ulp_bf16, ulp_e4m3
+from tests._util import ulp_bf16, ulp_e4m3
 
 D = 128
 DEV = "cuda"
@@ -73,55 +74,6 @@ def changed_pages(after: torch.Tensor, before: torch.Tensor, chunk=2048) -> set:
         d = (a[i:i + chunk] != b[i:i + chunk]).any(dim=1)
         out.append(torch.nonzero(d).flatten() + i)
     return set(torch.cat(out).tolist()) if out else set()
-
-
-U32 = 2.0 ** -24
-# Relative bound on the difference of the RMSNorm output y between two fp32
-# evaluations that sum the 128 squares in different orders (sequential: gamma_127,
-# 16-term lanes + 3-level tree: gamma_18; halved by the square root), plus the
-# roundings of +eps and the two products on each side, the correctly rounded
-# sqrt and 1/x of the definition (u each) and the kernel's rsqrtf (at most 2
-# ulp, 4 u): see the parity section of the design notes.  The rotation then
-# adds at most 2 u of each product term.
-K_COND = 87.0
-
-
-def _spacing_bf16(v):
-    v = np.abs(np.asarray(v, np.float64))
-    e = np.floor(np.log2(np.maximum(v, 2.0 ** -133)))
-    return 2.0 ** (np.maximum(e, -126) - 7)
-
-
-def _spacing_e4m3(v):
-    v = np.abs(np.asarray(v, np.float64))
-    e = np.floor(np.log2(np.maximum(v, 2.0 ** -9)))
-    return 2.0 ** (np.maximum(e, -6) - 3)
-
-
-def rotation_terms(w, r, head, pos):
-    """float64 |a c| + |b s| of every element's rotation pair (|y| outside the
-    rotated dims) for head `head` of packed row r at RoPE position pos."""
-    x = bf16_bits_to_f32(w.qkv[r, head * D:(head + 1) * D]).astype(np.float64)
-    wts = w.q_norm_w if head < w.Hq else w.k_norm_w
-    if wts is not None:
-        wf = bf16_bits_to_f32(wts).astype(np.float64)
-        if w.norm_style == 1:         # Gemma-style: 1 + w
-            wf = 1.0 + wf
-        y = x / np.sqrt(np.mean(x * x) + w.eps) * wf
-    else:
-        y = x
-    half = w.rot_dim // 2
-    c = np.abs(w.cos_sin[pos, :half].astype(np.float64))
-    sn = np.abs(w.cos_sin[pos, half:w.rot_dim].astype(np.float64))
-    t = np.abs(y).copy()
-    if w.rope_style == 0:
-        i0, i1 = np.arange(half), np.arange(half) + half
-    else:
-        i0, i1 = 2 * np.arange(half), 2 * np.arange(half) + 1
-    tp = np.abs(y[i0]) * c + np.abs(y[i1]) * sn
-    t[i0] = tp
-    t[i1] = tp
-    return t
 
 
 class AppendRun:
@@ -246,7 +198,7 @@ class AppendRun:
             return float(qs[b, h, r - int(self.q_indptr[b])])
         return float(qs[r, h])
 
-    def check(self, ref=None, *, exact_frac_min=0.99):
+    def check(self, ref=None):
         """Compare the device state with the oracle; returns a small report."""
         w = self.w
         ref = self.run_oracle() if ref is None else ref
@@ -278,7 +230,7 @@ class AppendRun:
             assert np.array_equal(ovg, ref["out_v"]), "owned V rows"
             ulp = ulp_bf16 if w.kv_esize == 2 else ulp_e4m3
             d = ulp(og, ref["out_k"])
-            rep["k_cond"] = self._conditioned(d, og, ref["out_k"], ref, "k_owned")
+            assert d.max() <= 1, f"owned K: max ulp {d.max()}"
             rep["k_exact_frac"] = float((d == 0).mean())
         # touched pages
         inner = w.page_size * w.Hkv * D
@@ -292,15 +244,14 @@ class AppendRun:
             ulp = ulp_bf16 if w.kv_esize == 2 else ulp_e4m3
             d = ulp(kg, ref["k"])
             d = np.where(kmask, d, 0)
-            rep["k_cond"] = self._conditioned(d, kg, ref["k"], ref, "k")
+            assert d.max() <= 1, f"K rows: max ulp {d.max()}"
             rep["k_exact_frac"] = float((d[kmask] == 0).mean()) if kmask.any() else 1.0
         # out_q
         oq = _np(self.out_q)
         if w.T:
             d = (ulp_bf16 if w.q_esize == 2 else ulp_e4m3)(oq, ref["out_q"])
-            rep["q_cond"] = self._conditioned(d, oq, ref["out_q"], ref, "q")
+            assert d.max() <= 1, f"out_q: max ulp {d.max()}"
             rep["q_exact_frac"] = float((d == 0).mean())
-            assert rep["q_exact_frac"] >= exact_frac_min, rep
             if w.quant_policy == 1:
                 qs = self.q_scale.cpu().numpy()
                 want = ref["q_scale"]
@@ -310,61 +261,9 @@ class AppendRun:
                 rel = np.abs(qs[m] - want[m]) / np.abs(want[m])
                 assert rel.max() <= 1e-5, f"q_scale rel {rel.max()}"
                 rep["q_scale_rel_max"] = float(rel.max())
+                rep["q_scale_exact_frac"] = float(
+                    (qs[m].view(np.uint32) == want[m].view(np.uint32)).mean())
         return rep
-
-    def _conditioned(self, d, got, want, ref, which):
-        """Elements more than 1 ulp apart must be within the propagated bound
-        1 spacing + K_COND * u * (|a c| + |b s|) (scaled into payload units).
-        Returns how many elements needed that clause."""
-        w = self.w
-        idx = np.argwhere(d > 1)
-        if idx.size == 0:
-            return 0
-        bf = (w.q_esize if which == "q" else w.kv_esize) == 2
-        dec = bf16_bits_to_f32 if bf else e4m3_decode
-        spacing = _spacing_bf16 if bf else _spacing_e4m3
-        tokmap = self._k_token_map(ref) if which == "k" else None
-        bad = []
-        for ix in idx:
-            if which == "q":
-                r, h, i = (int(v) for v in ix)
-                head = h
-            elif which == "k_owned":           # out_k [T, Hkv, 128]
-                r, kh, i = (int(v) for v in ix)
-                head = w.Hq + kh
-            else:
-                pg, row, kh, i = (int(v) for v in ix)
-                r = tokmap[(pg, row)]
-                head = w.Hq + kh
-            b = int(np.searchsorted(self.q_indptr, r, side="right") - 1)
-            pos = int(w.positions[r]) if w.positions is not None else \
-                r + int(self.seq_lens[b]) - int(self.q_indptr[b + 1])
-            t = rotation_terms(w, r, head, pos)[i]
-            if which == "q":
-                scale = {0: 1.0, 2: w.q_scale_inv}.get(w.quant_policy)
-                if scale is None:
-                    scale = 1.0 / self.q_scale_at(ref["q_scale"], r, h)
-            else:
-                scale = 1.0 if w.quant_policy == 0 else 1.0 / w.k_scale
-            g = float(dec(np.array([got[tuple(ix)]]))[0])
-            o = float(dec(np.array([want[tuple(ix)]]))[0])
-            tol = max(float(spacing(g)), float(spacing(o))) + K_COND * U32 * t * scale
-            if not abs(g - o) <= tol:
-                bad.append((tuple(int(v) for v in ix), g, o, t, int(d[tuple(ix)])))
-        assert not bad, f"{which}: {len(bad)} elements beyond the bound, e.g. {bad[:4]}"
-        assert len(idx) <= max(2, 1e-3 * d.size), f"{which}: too many >1 ulp elements {len(idx)}"
-        return int(len(idx))
-
-    def _k_token_map(self, ref):
-        w = self.w
-        P = w.page_size
-        remap = {g: i for i, g in enumerate(ref["pages"])}
-        out = {}
-        for b in range(w.B):
-            lo, hi, L = int(self.q_indptr[b]), int(self.q_indptr[b + 1]), int(self.seq_lens[b])
-            for p in range(L - (hi - lo), L):
-                out[(remap[int(w.page_table[b, p // P])], p % P)] = lo + p - (L - (hi - lo))
-        return out
 
     def _k_written_rows(self, ref):
         """bool mask over the compact K image: rows written by new tokens."""

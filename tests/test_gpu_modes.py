@@ -28,7 +28,12 @@ SCHEDULES = [1, 2]
 def check(w, **kw):
     r = AppendRun(w, **kw)
     r.launch()
-    return r, r.check(exact_frac_min=0.95)
+    rep = r.check()
+    if not rep.get("flagged"):
+        # the same correctly rounded steps on both sides: bit-identical
+        assert rep.get("q_exact_frac", 1.0) == 1.0 and rep.get("k_exact_frac", 1.0) == 1.0, rep
+        assert rep.get("q_scale_exact_frac", 1.0) == 1.0, rep
+    return r, rep
 
 
 # ------------------------------------------------------ prefill q_scale layout
