@@ -375,7 +375,7 @@ __device__ __forceinline__ int quad_kind(const HeadParams& a, int h0) {
 // squares is exact whenever its nonzero magnitudes span at most 2^15 -- so no
 // summation order (four lane chains, then the group's xor tree) can change
 // it.  One rounding to fp32, then +eps, the square root and the reciprocal,
-// each correctly rounded.
+// each correctly rounded (rn_recip_sqrt).
 __device__ __forceinline__ float inv_rms(const float2* y, float eps, unsigned gmask) {
   double s[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
@@ -389,7 +389,7 @@ __device__ __forceinline__ float inv_rms(const float2* y, float eps, unsigned gm
   ss += __shfl_xor_sync(gmask, ss, 2);
   ss += __shfl_xor_sync(gmask, ss, 1);
   const float ms = __double2float_rn(ss * (1.0 / kHeadDim));
-  return __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
+  return rn_recip_sqrt(__fadd_rn(ms, eps));
 }
 
 // Norm + RoPE + quantisation + store of head h of row r.  xa/xb: the lane's two
