@@ -3,24 +3,28 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one fused call (one kernel: validation, Q/K RMSNorm, RoPE,
+One step = one fused call (one kernel: validation, Q/K RMSNorm, RoPE, FP8
 quantisation, paged K/V scatter, last-page tail zeroing, flags) over one batch
-of the Qwen3-style decode workload: 128 requests x 1 new token, Hq 32 / Hkv 8,
-head_dim 128, page 16, 1M-slot BF16 NHD cache.  Inputs are synthetic and
-seeded (workloads.py).  Each step uses its own replica of the step inputs
-(packed QKV, metadata, page table, out_q) and writes pages of its own, with
-enough replicas that the per-step data rotated over in the timed region is
-larger than L2 (126 MB); the timed launches are replayed from CUDA graphs.
+of the ragged FP8 prefill workload: 16 requests with U[0, 2048] new tokens
+each (two empty; 9,212 tokens in all) on U[0, 4096] prior context, Hq 64 /
+Hkv 8, head_dim 128, page 16, static FP8 E4M3 Q/K/V.  Inputs are synthetic
+and seeded (workloads.py).  Each step uses its own replica of the step inputs
+(packed QKV, metadata, page table, out_q: the same token counts with other
+data, positions and pages), and a step's data (288 MB) is larger than L2
+(126 MB); the timed launches are replayed from CUDA graphs.
 
-Rank 0 prints one JSON line.  `value` = tokens/s over all ranks (the
-max-over-ranks device time of K steps); `roofline` = algorithmic bytes per
-launch / average launch time, against the measured HBM copy bandwidth;
-`e2e` = the same metric through the public API with pinned host buffers
-(host->device copies of the step's inputs and device->host copies of out_q
-and flags inside the timed region); `cpu_baseline` = the CPU oracle on a
-bounded sample, single-threaded (`cpu_baseline_all_cores`: one process per
-host core on disjoint requests); `per_config` adds the other named workloads (kernel time,
-GB/s, fraction of peak) measured the same way, outside the timed region.
+Rank 0 prints one JSON line.  The timed region (exactly K launches) is
+repeated; `ms_per_step` and `value` come from the median region.  `value` =
+tokens/s over all ranks (the max-over-ranks device time of a region);
+`roofline` = algorithmic bytes per launch / median launch time, against the
+measured HBM copy bandwidth; `e2e` = the same metric through the public API
+with pinned host buffers (host->device copies of the step's inputs and
+device->host copies of out_q and flags inside the timed region);
+`cpu_baseline` = the CPU oracle on a bounded sample, single-threaded
+(`cpu_baseline_all_cores`: one process per host core on disjoint requests);
+`per_config` (last, compact) adds every named workload measured the same way
+outside the timed region: microseconds per launch, fraction of the peak, and
+the two schedules forced.
 
 --impl reference times the CPU oracle (the reference arm of this build) on
 the host cores on the same workload, metric and unit.
@@ -48,15 +52,19 @@ import workloads  # noqa: E402
 METRIC = "fused QKnorm+RoPE+quant+paged-append tokens/s and HBM GB/s (% of peak), 1 B200"
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
-MAIN_WORKLOAD = "qwen3_decode_bf16"
+MAIN_WORKLOAD = "ragged_prefill_fp8"
+MIN_TIMED_LAUNCHES = 200
 FALLBACK_HBM_GBS = 6650.0
 
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200000)
-    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--repeats", type=int, default=None,
+                    help="timed regions of exactly --steps launches each (default: at least 5, "
+                         "and at least 200 launches in all); the median region is reported")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=MAIN_WORKLOAD, choices=sorted(workloads.APPEND_CONFIGS))
     ap.add_argument("--replicas", type=int, default=None, help="override the replica count")
@@ -66,7 +74,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU budget of the oracle baseline sample")
-    ap.add_argument("--e2e-steps", type=int, default=3000)
+    ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--profile", action="store_true",
                     help="profiling run: only --workload (or mla_decode), --steps eager launches, "
                          "no graphs, no e2e / per-config / CPU legs, no JSON line")
@@ -122,24 +130,32 @@ def kernel_source_hash(names=APPEND_KERNEL_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "traffic.json")
+
+
 def profiled_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary of this workload,
-    if it was captured on the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", f"append_paged_{workload}.md")
-    if not os.path.exists(path):
-        return None
-    vals = {}
-    with open(path) as f:
-        for line in f:
-            if line.startswith("bench-key:"):
-                k, _, v = line[len("bench-key:"):].strip().partition("=")
-                vals[k.strip()] = v.strip()
-    if vals.get("kernel_sources") != kernel_source_hash():
-        return None
+    """Measured memory traffic per launch of this workload's kernel, from the
+    committed ncu record profiles/traffic.json, if it was captured on the
+    current append-kernel sources.  Returns (traffic bytes or None, details).
+
+    traffic = dram__bytes_read.sum + 32 x lts__t_sectors_op_write.sum: reads
+    counted at DRAM, writes where they enter L2 (a write-back cache: a
+    launch's last writes are still in L2 when it ends, so dram__bytes_write
+    undercounts them; every sector written reaches DRAM once)."""
     try:
-        return int(vals["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None, {"note": "no traffic record"}
+    if rec.get("kernel_sources") != kernel_source_hash():
+        return None, {"note": "traffic record taken on other kernel sources"}
+    e = rec.get("workloads", {}).get(workload)
+    if not e:
+        return None, {"note": f"no traffic record for {workload}"}
+    t = int(e["dram_read_bytes"]) + int(e["l2_write_bytes"])
+    return t, {"dram_read": int(e["dram_read_bytes"]), "l2_write": int(e["l2_write_bytes"]),
+               "dram_write": int(e["dram_write_bytes"]),
+               "basis": "ncu: dram__bytes_read.sum + 32 x lts__t_sectors_op_write.sum per launch"}
 
 
 class ClockSampler:
@@ -211,6 +227,31 @@ def gpu_smi_id(torch, dev) -> str:
 
 # -------------------------------------------------------- device workloads
 
+def replica_workloads(name, min_bytes=3 * L2_BYTES, max_replicas=64, seed_offset=0,
+                      small_cache=False):
+    """The replicas a bench of workload `name` rotates over: enough that one
+    cycle moves at least `min_bytes` (at least 2, at most `max_replicas`).
+    Replica r is the workload drawn with seed base + seed_offset + 7919 r; a
+    workload that draws its token counts (the ragged prefill) keeps the first
+    replica's counts, so that every step has the same tokens and shape."""
+    make = workloads.APPEND_CONFIGS[name]
+    if small_cache:
+        def make(seed=None, _f=workloads.APPEND_CONFIGS[name], **kw):
+            return workloads.shrink_cache(_f(**kw) if seed is None else _f(seed=seed, **kw))
+    base = make()
+    per = workloads.append_bytes(base)["total"]
+    R = int(min(max_replicas, max(2, math.ceil(min_bytes / per))))
+    base_n = np.diff(base.q_indptr)
+    ws = []
+    for r in range(R):
+        sd = base.seed + seed_offset + 7919 * r
+        rep = base if sd == base.seed else make(seed=sd)
+        if rep.T != base.T:
+            rep = make(seed=sd, n_new=base_n)
+        ws.append(rep)
+    return ws
+
+
 class AppendBench:
     """R replicas of one append workload sharing one pair of KV caches."""
 
@@ -218,18 +259,10 @@ class AppendBench:
                  seed_offset=0, schedule=0, small_cache=False):
         self.torch, self.fqr, self.dev = torch, fqr, device
         self.schedule = schedule
-        make = workloads.APPEND_CONFIGS[name]
-        if small_cache:
-            def make(seed=None, _f=workloads.APPEND_CONFIGS[name]):
-                return workloads.shrink_cache(_f() if seed is None else _f(seed=seed))
-        base = make()
+        ws = replica_workloads(name, min_bytes, max_replicas, seed_offset, small_cache)
+        self.R = len(ws)
+        base = ws[0]
         self.name = base.name
-        per = workloads.append_bytes(base)["total"]
-        self.R = int(min(max_replicas, max(2, math.ceil(min_bytes / per))))
-        ws = []
-        for r in range(self.R):
-            sd = base.seed + seed_offset + 7919 * r
-            ws.append(base if sd == base.seed else make(seed=sd))
         self.ws = ws
         self.bytes = [workloads.append_bytes(w)["total"] for w in ws]
         self.T = base.T
@@ -346,10 +379,13 @@ class MlaBench:
             raise self.fqr.FqrError(rc)
 
 
-def time_launches(torch, bench, steps, warmup, graph_chunk=1000, barrier=None, marks=None):
-    """Warm up, then time exactly `steps` launches (replayed from CUDA graphs
-    of up to `graph_chunk` launches, cycling over the replicas) with CUDA
-    events on the launching stream.  Returns (elapsed_ms, bytes)."""
+def time_launches(torch, bench, steps, warmup, repeats=1, graph_chunk=1000, barrier=None,
+                  marks=None):
+    """Warm up, then time `repeats` regions of exactly `steps` launches each
+    (replayed from CUDA graphs of up to `graph_chunk` launches, cycling over
+    the replicas) with CUDA events on the launching stream, each region
+    bracketed by a barrier and a device synchronisation.  Returns (the list of
+    region times in ms, the algorithmic bytes of one region)."""
     stream = torch.cuda.current_stream()
     h = stream.cuda_stream
     for i in range(warmup):
@@ -372,32 +408,35 @@ def time_launches(torch, bench, steps, warmup, graph_chunk=1000, barrier=None, m
     g_full = capture(chunk, 0) if full else None
     g_rest = capture(rest, 0) if rest else None
     # replay once untimed (graph upload)
-    if g_full is not None:
-        g_full.replay()
+    for g in (g_full, g_rest):
+        if g is not None:
+            g.replay()
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    if barrier is not None:
-        barrier()
-    torch.cuda.synchronize()
     if marks is not None:
         marks(True)
-    start.record(stream)
-    for _ in range(full):
-        g_full.replay()
-    if g_rest is not None:
-        g_rest.replay()
-    end.record(stream)
-    torch.cuda.synchronize()
+    times = []
+    for _ in range(repeats):
+        if barrier is not None:
+            barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(full):
+            g_full.replay()
+        if g_rest is not None:
+            g_rest.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+        if barrier is not None:
+            barrier()
+        times.append(start.elapsed_time(end))
     if marks is not None:
         marks(False)
-    if barrier is not None:
-        barrier()
-    ms = start.elapsed_time(end)
     nbytes = sum(bench.bytes[i % bench.R] for i in range(chunk)) * full + \
         sum(bench.bytes[i % bench.R] for i in range(rest))
     del g_full, g_rest
-    return ms, nbytes
+    return times, nbytes
 
 
 def e2e_measure(torch, fqr, bench, steps):
@@ -606,7 +645,10 @@ def config_block(w, bench):
          "io_dtype": "bf16 in, " + ("bf16" if w.quant_policy == 0 else "e4m3") + " out",
          "parallelism": "replicas"}
     if bench is not None:
+        seeds = sorted({x.seed for x in bench.ws})
         c["replicas"] = bench.R
+        c["seeds"] = (f"{seeds[0]} (+7919 per replica): workload draws; the replicas keep the "
+                      f"first one's token counts" if len(seeds) > 1 else str(seeds[0]))
         c["l2"] = (f"inputs larger than L2: each step uses its own replica of the step inputs "
                    f"({bench.R} replicas, {sum(bench.bytes) / 1e6:.0f} MB rotated per cycle)")
     return c
@@ -643,24 +685,28 @@ def main(argv=None):
     peak, peak_src = load_peaks()
     bench = AppendBench(args.workload, torch, fqr, dev, seed_offset=1000 * rank,
                         schedule=args.schedule)
+    repeats = args.repeats or max(5, math.ceil(MIN_TIMED_LAUNCHES / max(args.steps, 1)))
     sampler = ClockSampler(gpu_smi_id(torch, dev)) if rank == 0 else None
     if sampler is not None:
         time.sleep(1.0)   # let nvidia-smi start sampling before the warm-up
-    ms, nbytes = time_launches(torch, bench, args.steps, args.warmup, barrier=barrier,
-                               marks=sampler.mark if sampler else None)
+    region_ms, nbytes = time_launches(torch, bench, args.steps, args.warmup, repeats=repeats,
+                                      barrier=barrier, marks=sampler.mark if sampler else None)
     bench.check_flags()
     clocks = sampler.stop() if sampler else None
-    ms_max = max_over_ranks(torch, dist, ms, dev)
+    region_max = [max_over_ranks(torch, dist, m, dev) for m in region_ms]
+    ms_max = statistics.median(region_max)
+    ms_local = statistics.median(region_ms)
     value = world * bench.T * args.steps / (ms_max / 1e3)
-    per_launch_s = ms / 1e3 / args.steps
+    per_launch_s = ms_local / 1e3 / args.steps
     achieved = nbytes / args.steps / per_launch_s / 1e9
+    traffic, traffic_parts = profiled_traffic(args.workload)
 
     e2e = e2e_measure(torch, fqr, bench, min(args.e2e_steps, max(args.steps, 1)))
     e2e_ms = max_over_ranks(torch, dist, e2e["ms_per_step"], dev)
     e2e["value"] = world * bench.T / (e2e_ms / 1e3)
     per_config = None
     if rank == 0 and not args.no_per_config:
-        per_config = measure_per_config(torch, fqr, dev, peak, args.workload)
+        per_config = measure_per_config(torch, fqr, dev, peak)
     cpu = cpu_all = None
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         cpu = cpu_baseline(bench.ws[0], args.cpu_seconds)
@@ -670,19 +716,25 @@ def main(argv=None):
         dist.destroy_process_group()
     if rank != 0:
         return 0
+    us = [m * 1e3 / args.steps for m in region_ms]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "gpu_launches": args.steps,
         "config": config_block(bench.ws[0], bench),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
-                     "peak_source": peak_src,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "traffic_over_algorithmic": (traffic / (nbytes / args.steps)
+                                                  if traffic else None),
                      "bytes_per_launch": nbytes / args.steps,
-                     "kernel": describe_plan(fqr.append_plan(bench.reps[0]["params"])),
-                     "timing": "CUDA events around graph "
-                     "replays of back-to-back launches; average launch = region / steps"},
-        "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks, "cpu_baseline": cpu,
+                     "us_per_launch": per_launch_s * 1e6,
+                     "timing": f"median of {repeats} regions of exactly {args.steps} launches "
+                               f"(CUDA events, CUDA-graph replays of back-to-back launches); "
+                               f"region us/launch min {min(us):.2f} max {max(us):.2f}",
+                     "peak_source": peak_src, "traffic_parts": traffic_parts,
+                     "kernel": describe_plan(fqr.append_plan(bench.reps[0]["params"]))},
+        "e2e": e2e, "clocks": clocks, "cpu_baseline": cpu,
         "cpu_baseline_all_cores": cpu_all,
         "per_config": per_config,
     }
@@ -708,36 +760,41 @@ def run_profile(args, torch, fqr, dev):
     return 0
 
 
-def measure_per_config(torch, fqr, dev, peak, main_name, steps=20000, warmup=200):
+def _short(x, digits=3):
+    return float(f"{x:.{digits}g}")
+
+
+def measure_per_config(torch, fqr, dev, peak, warmup=50, repeats=3):
+    """Every named workload, timed like the headline (median of `repeats`
+    regions), in a compact form: us = microseconds per launch (automatic
+    schedule), frac = algorithmic bytes / time / peak, lat / str = us per
+    launch with the latency / streaming schedule forced, MB = algorithmic
+    megabytes per launch, T = tokens per launch."""
     out = {}
+
+    def timed(b):
+        n = max(200, min(4000, int(4e9 / max(b.bytes))))
+        reg, nbytes = time_launches(torch, b, n, warmup, repeats=repeats)
+        return statistics.median(reg) * 1e3 / n, nbytes / n
+
     for name in sorted(workloads.APPEND_CONFIGS):
         b = AppendBench(name, torch, fqr, dev)
-        n = max(200, min(steps, int(2e10 / max(b.bytes))))   # ~a few hundred ms each
-        ms, nbytes = time_launches(torch, b, n, warmup)
+        us, per = timed(b)
         b.check_flags()
-        us = ms * 1e3 / n
-        gbs = nbytes / n / (us * 1e-6) / 1e9
-        out[name] = {"workload": b.name, "us_per_launch": us, "tokens_per_s": b.T / (us * 1e-6),
-                     "GB_per_s": gbs, "frac_of_peak": gbs / peak,
-                     "bytes_per_launch": nbytes / n, "replicas": b.R, "launches": n,
-                     "us_per_launch_by_schedule": {}}
-        for sched, label in ((1, "latency"), (2, "streaming")):   # both schedules, for tuning
+        e = {"us": _short(us), "frac": _short(per / (us * 1e-6) / 1e9 / peak),
+             "MB": _short(per / 1e6), "T": b.T}
+        for sched, label in ((1, "lat"), (2, "str")):   # both schedules, for tuning
             for st in b.reps:
                 st["params"].schedule = sched
-            ms_s, _ = time_launches(torch, b, n, warmup)
-            out[name]["us_per_launch_by_schedule"][label] = ms_s * 1e3 / n
+            e[label] = _short(timed(b)[0])
+        out[name] = e
         del b
         torch.cuda.empty_cache()
     for name in workloads.MLA_CONFIGS:
         m = MlaBench(torch, fqr, dev, name=name)
-        n = 20000
-        ms, nbytes = time_launches(torch, m, n, warmup)
-        us = ms * 1e3 / n
-        gbs = nbytes / n / (us * 1e-6) / 1e9
-        out[name] = {"workload": m.name, "us_per_launch": us,
-                     "tokens_per_s": m.T / (us * 1e-6), "GB_per_s": gbs,
-                     "frac_of_peak": gbs / peak, "bytes_per_launch": nbytes / n,
-                     "replicas": m.R, "launches": n}
+        us, per = timed(m)
+        out[name] = {"us": _short(us), "frac": _short(per / (us * 1e-6) / 1e9 / peak),
+                     "MB": _short(per / 1e6), "T": m.T}
         del m
         torch.cuda.empty_cache()
     return out

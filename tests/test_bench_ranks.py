@@ -87,3 +87,47 @@ def test_describe_plan_names_the_schedule_and_variants():
     d = bench.describe_plan(dict(schedule=2, grid=296, block_threads=288, tasks=9212,
                                  warp_check=0, bulk_tails=0, request_tails=0))
     assert "streaming schedule" in d and "296 blocks of 288 threads" in d and "9212 units" in d
+
+
+def test_prefill_replicas_keep_the_batch_shape():
+    """Every replica of the headline workload has the same tokens per request
+    (so every timed step does the same work) but its own positions, pages and
+    data; bytes per launch stay within a fraction of a percent."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    import workloads
+    ws = bench.replica_workloads("ragged_prefill_fp8", min_bytes=1, max_replicas=2)
+    assert len(ws) == 2
+    a, b = ws
+    assert a.T == b.T and np.array_equal(a.q_indptr, b.q_indptr)
+    assert not np.array_equal(a.seq_lens, b.seq_lens)
+    assert not np.array_equal(a.page_table, b.page_table)
+    assert not np.array_equal(a.qkv[:4], b.qkv[:4])
+    ba, bb = (workloads.append_bytes(w)["total"] for w in ws)
+    assert abs(ba - bb) / ba < 1e-3
+    # decode workloads keep one token per request in every replica
+    ds = bench.replica_workloads("qwen3_decode_bf16", min_bytes=1, max_replicas=3)
+    assert len(ds) == 2 and {w.T for w in ds} == {128}
+
+
+def test_traffic_record_needs_the_current_kernel_sources(tmp_path, monkeypatch):
+    """The traffic figure is used only when the ncu record was taken on the
+    sources the library is built from now."""
+    import json
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    rec = {"kernel_sources": bench.kernel_source_hash(),
+           "workloads": {"ragged_prefill_fp8": {"dram_read_bytes": 100, "l2_write_bytes": 50,
+                                                "dram_write_bytes": 40}}}
+    path = tmp_path / "traffic.json"
+    path.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "TRAFFIC_RECORD", str(path))
+    t, parts = bench.profiled_traffic("ragged_prefill_fp8")
+    assert t == 150 and parts["dram_write"] == 40
+    assert bench.profiled_traffic("qwen3_decode_bf16")[0] is None
+    rec["kernel_sources"] = "0" * 16
+    path.write_text(json.dumps(rec))
+    assert bench.profiled_traffic("ragged_prefill_fp8")[0] is None
