@@ -342,7 +342,8 @@ class MlaBench:
                                                cos_sin_rows=base.cos_sin_rows,
                                                q_quant=base.q_quant,
                                                q_scale_inv=base.q_scale_inv,
-                                               upper_max=base.upper_max)
+                                               upper_max=base.upper_max,
+                                               q_group=base.q_group)
                             for r in range(1, self.R)]
         self.bytes = [workloads.mla_bytes(w)["total"] for w in self.ws]
         self.T = base.T
@@ -361,10 +362,9 @@ class MlaBench:
             if w.q_quant:   # Q quantised into q_out / q_scale (q read-only)
                 q_out = torch.empty((w.T, w.Hq, w.nope_dim + w.rope_dim), dtype=torch.uint8,
                                     device=device)
-                q_scale = torch.empty({2: (w.T,), 3: (w.T, w.Hq)}.get(w.q_quant, (1,)),
-                                      dtype=torch.float32, device=device)
+                q_scale = torch.empty(w.q_scale_shape, dtype=torch.float32, device=device)
                 qq = dict(q_quant=w.q_quant, q_scale_inv=self.qsi, upper_max=w.upper_max,
-                          q_out=q_out, q_scale=q_scale)
+                          q_out=q_out, q_scale=q_scale, q_group=w.q_group)
             self.keep.append((q, kv_c, k_pe, ind, sl, bt, flags, qq))
             self.params.append(fqr.mla_params(q, kv_c, k_pe, self.cs, ind, sl, bt, self.latent,
                                               flags, nope_dim=w.nope_dim,

@@ -79,6 +79,9 @@ extern "C" {
  *     y = x * (1/sqrt(sum(x^2)/128 + eps)) * w         (Q heads with q_norm_w,
  *                                                       K heads with k_norm_w;
  *                                       w -> 1 + w for norm_style GEMMA)
+ *            the mean square sum(x^2)/128 is the fp32 rounding of the exact
+ *            mean of the squares (no summation order enters); + eps, the
+ *            square root and the reciprocal are each correctly rounded
  *     NeoX:  (y_i, y_{i+64})  -> (y_i c_i - y_{i+64} s_i, y_{i+64} c_i + y_i s_i)
  *     GPT-J: (y_2i, y_2i+1)   -> (y_2i c_i - y_2i+1 s_i, y_2i+1 c_i + y_2i s_i)
  *            with c_i = cos_sin[pos, i], s_i = cos_sin[pos, rot_dim/2 + i];
@@ -281,9 +284,17 @@ int fqr_pipeline_destroy(fqr_pipeline* p);
  *                       1e-6) / upper_max, q_scale[r] = s         (fp32 [T])
  *   FQR_MLA_Q_HEAD:     the same with the max over head h alone,
  *                       q_scale[r * Hq + h] = s                   (fp32 [T, Hq])
+ *   FQR_MLA_Q_GROUP:    the same with the max over each group of q_group
+ *                       consecutive values of v of one head (block
+ *                       quantisation; the last group of a head is shorter
+ *                       when q_group does not divide nope + rope; q_group
+ *                       >= nope + rope gives one group per head),
+ *                       q_scale[(r * Hq + h) * NG + k] = s of group k,
+ *                       NG = ceil((nope + rope) / q_group)  (fp32 [T, Hq, NG])
  *
  * Constraints: rope_dim == 64; nope_dim, q_token_stride, q_head_stride
- * multiples of 4 (of 8, and nope_dim <= 256, with Q quantisation);
+ * multiples of 4 (of 8, and nope_dim <= 256, with Q quantisation); q_group
+ * (FQR_MLA_Q_GROUP) a multiple of 8, at least 8;
  * kv_lora_rank, kv_c_stride
  * multiples of 8; k_pe_stride a multiple of 4; q, kv_c, k_pe, latent_cache,
  * q_out 16-byte aligned.
@@ -292,6 +303,7 @@ int fqr_pipeline_destroy(fqr_pipeline* p);
 #define FQR_MLA_Q_STATIC 1
 #define FQR_MLA_Q_TOKEN 2
 #define FQR_MLA_Q_HEAD 3
+#define FQR_MLA_Q_GROUP 4
 typedef struct fqr_mla_params {
   uint16_t* q;                 /* bf16, element (r, h, d) at
                                   r*q_token_stride + h*q_head_stride + d     */
@@ -318,7 +330,8 @@ typedef struct fqr_mla_params {
   const float* q_scale_inv;    /* device fp32 scalar (FQR_MLA_Q_STATIC)      */
   float upper_max;             /* dynamic modes: finite, in (0, 448]         */
   void* q_out;                 /* e4m3 [T, Hq, nope + rope] (q_quant != 0)   */
-  float* q_scale;              /* fp32 [T] or [T, Hq] (dynamic modes)        */
+  float* q_scale;              /* fp32 [T], [T, Hq] or [T, Hq, NG] (dynamic) */
+  int32_t q_group;             /* values per group (FQR_MLA_Q_GROUP)         */
 } fqr_mla_params;
 
 int fqr_concat_mla_cache(const fqr_mla_params* p, void* stream);

@@ -28,7 +28,7 @@ FQR_OK, FQR_EINVAL, FQR_ENOTSUP, FQR_ECUDA = 0, 1, 2, 3
 SCHEDULE_AUTO, SCHEDULE_LATENCY, SCHEDULE_STREAMING = 0, 1, 2
 FLAG_TIMEOUT = -2
 NORM_RMS, NORM_GEMMA = 0, 1
-MLA_Q_NONE, MLA_Q_STATIC, MLA_Q_TOKEN, MLA_Q_HEAD = 0, 1, 2, 3
+MLA_Q_NONE, MLA_Q_STATIC, MLA_Q_TOKEN, MLA_Q_HEAD, MLA_Q_GROUP = 0, 1, 2, 3, 4
 HEAD_DIM = 128
 MAX_BATCH = 16384
 
@@ -72,7 +72,7 @@ class MlaParams(ctypes.Structure):
         ("latent_cache", c_vp), ("num_blocks", c_i32), ("block_size", c_i32),
         ("cache_fp8", c_i32), ("kv_scale", c_vp), ("flags", c_vp),
         ("q_quant", c_i32), ("q_scale_inv", c_vp), ("upper_max", c_f32),
-        ("q_out", c_vp), ("q_scale", c_vp),
+        ("q_out", c_vp), ("q_scale", c_vp), ("q_group", c_i32),
     ]
 
 
@@ -352,7 +352,8 @@ class StagedAppend:
 def mla_params(q, kv_c, k_pe, cos_sin_cache, q_indptr, seq_lens, block_table, latent_cache,
                flags, *, nope_dim: int, rope_style: int = 1, kv_scale=None,
                positions=None, q_quant: int = MLA_Q_NONE, q_scale_inv=None,
-               upper_max: float = 448.0, q_out=None, q_scale=None) -> MlaParams:
+               upper_max: float = 448.0, q_out=None, q_scale=None,
+               q_group: int = 0) -> MlaParams:
     T = int(q.shape[0])
     rope_dim = int(k_pe.shape[1]) if k_pe.dim() == 2 else 0
     return MlaParams(
@@ -367,7 +368,8 @@ def mla_params(q, kv_c, k_pe, cos_sin_cache, q_indptr, seq_lens, block_table, la
         num_blocks=int(latent_cache.shape[0]), block_size=int(latent_cache.shape[1]),
         cache_fp8=1 if latent_cache.element_size() == 1 else 0, kv_scale=_ptr(kv_scale),
         flags=_ptr(flags), q_quant=int(q_quant), q_scale_inv=_ptr(q_scale_inv),
-        upper_max=float(upper_max), q_out=_ptr(q_out), q_scale=_ptr(q_scale))
+        upper_max=float(upper_max), q_out=_ptr(q_out), q_scale=_ptr(q_scale),
+        q_group=int(q_group))
 
 
 def concat_mla_cache(q, kv_c, k_pe, cos_sin_cache, q_indptr, seq_lens, block_table,
@@ -390,4 +392,5 @@ __all__ = ["LIB", "LIB_PATH", "AppendParams", "MlaParams", "FqrError", "strerror
            "concat_mla_cache", "concat_mla_cache_raw", "FQR_OK", "FQR_EINVAL",
            "FQR_ENOTSUP", "FQR_ECUDA", "HEAD_DIM", "MAX_BATCH", "SCHEDULE_AUTO",
            "SCHEDULE_LATENCY", "SCHEDULE_STREAMING", "FLAG_TIMEOUT", "NORM_RMS",
-           "NORM_GEMMA", "MLA_Q_NONE", "MLA_Q_STATIC", "MLA_Q_TOKEN", "MLA_Q_HEAD"]
+           "NORM_GEMMA", "MLA_Q_NONE", "MLA_Q_STATIC", "MLA_Q_TOKEN", "MLA_Q_HEAD",
+           "MLA_Q_GROUP"]

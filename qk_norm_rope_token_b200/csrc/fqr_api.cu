@@ -109,7 +109,8 @@ int check_mla(const fqr_mla_params* p) {
     if (p->q_token_stride < static_cast<int64_t>(p->Hq) * p->q_head_stride) return FQR_EINVAL;
     if (p->kv_c_stride < p->kv_lora_rank || p->k_pe_stride < p->rope_dim) return FQR_EINVAL;
   }
-  if (p->q_quant < FQR_MLA_Q_NONE || p->q_quant > FQR_MLA_Q_HEAD) return FQR_EINVAL;
+  if (p->q_quant < FQR_MLA_Q_NONE || p->q_quant > FQR_MLA_Q_GROUP) return FQR_EINVAL;
+  if (p->q_quant == FQR_MLA_Q_GROUP && (p->q_group < 8 || p->q_group % 8)) return FQR_EINVAL;
   if (p->q_quant != FQR_MLA_Q_NONE) {
     if (p->T > 0 && (!p->q_out || !aligned(p->q_out, 16))) return FQR_EINVAL;
     if (p->q_quant == FQR_MLA_Q_STATIC && !p->q_scale_inv) return FQR_EINVAL;

@@ -79,9 +79,7 @@ __device__ __forceinline__ float4 ld_smem_f4(const float* p) {
   return *reinterpret_cast<const float4*>(p);
 }
 
-__device__ void report_timeout(const PipeArgs& a) {
-  for (int b = threadIdx.x & 31; b < a.B; b += 32) a.flags[b] = kFlagTimeout;
-}
+__device__ void report_timeout(const PipeArgs& a) { flag_timeout(a.flags, a.B, threadIdx.x & 31); }
 
 // Unit u: packed row t, heads [h0, h0 + nh).
 __device__ __forceinline__ void unit_heads(const PipeArgs& a, int64_t u, int& t, int& h0,

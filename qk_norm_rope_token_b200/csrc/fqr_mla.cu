@@ -54,6 +54,8 @@ struct MlaArgs {
   float upper_max;
   unsigned char* q_out;
   float* q_scale;
+  int q_ng;      // per-group Q scales: groups per head, ceil((nope + 64) / q_group)
+  FastDiv gdiv;  // division by q_group
 };
 
 __device__ __forceinline__ uint2 ld_v2(const void* p) {
@@ -380,7 +382,93 @@ __device__ __forceinline__ void store_q_head(QHead& v, unsigned char* op, int no
   st_u32(op + nope + kRope / 2 + 4 * l8, pack4_e4m3(v.y + 4));
 }
 
-// Static and per-head scales: persistent warp tasks [latent rows | row x quad].
+// Per-group scales (FQR_MLA_Q_GROUP): groups of q_group consecutive values of
+// a head's v = [nope | rope(rope part)].  Each of the lane's runs -- its nope
+// chunks l8 + 8k (8 values) and its two 4-value rope runs -- lies inside one
+// group: q_group is a multiple of 8, nope a multiple of 8, and every run
+// starts on a multiple of 4 inside an 8-aligned block.  The groups' maxima
+// are reduced one group at a time over the head's 8 lanes; lane k % 8 stores
+// the scale of group k.
+constexpr int kRuns = kMaxChunks + 2;
+struct RunScales {
+  float sc[kRuns], rc[kRuns];
+};
+
+__device__ __forceinline__ void group_scales(const MlaArgs& a, const QHead& v, int l8,
+                                             unsigned gmask, float* qs, RunScales& rs) {
+  float m[kRuns];
+  int grp[kRuns];
+#pragma unroll
+  for (int k = 0; k < kMaxChunks; ++k) {
+    const int c = l8 + 8 * k;
+    m[k] = 0.0f;
+    grp[k] = -1;
+    if (c < a.nope / 8) {
+      float x[8];
+      unpack8(v.nope[k], x);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m[k] = fmaxf(m[k], fabsf(x[j]));
+      grp[k] = static_cast<int>(a.gdiv.div(static_cast<uint32_t>(8 * c)));
+    }
+  }
+  m[kMaxChunks] = fmaxf(fmaxf(fabsf(v.y[0]), fabsf(v.y[1])), fmaxf(fabsf(v.y[2]), fabsf(v.y[3])));
+  m[kMaxChunks + 1] =
+      fmaxf(fmaxf(fabsf(v.y[4]), fabsf(v.y[5])), fmaxf(fabsf(v.y[6]), fabsf(v.y[7])));
+  grp[kMaxChunks] = static_cast<int>(a.gdiv.div(static_cast<uint32_t>(a.nope + 4 * l8)));
+  grp[kMaxChunks + 1] =
+      static_cast<int>(a.gdiv.div(static_cast<uint32_t>(a.nope + kRope / 2 + 4 * l8)));
+#pragma unroll
+  for (int r = 0; r < kRuns; ++r) rs.sc[r] = 1.0f;
+  for (int k = 0; k < a.q_ng; ++k) {
+    float mk = 0.0f;
+#pragma unroll
+    for (int r = 0; r < kRuns; ++r)
+      if (grp[r] == k) mk = fmaxf(mk, m[r]);
+    mk = fmaxf(mk, __shfl_xor_sync(gmask, mk, 4));
+    mk = fmaxf(mk, __shfl_xor_sync(gmask, mk, 2));
+    mk = fmaxf(mk, __shfl_xor_sync(gmask, mk, 1));
+    const float sk = __fdiv_rn(fmaxf(mk, 1e-6f), a.upper_max);
+    if (l8 == (k & 7)) qs[k] = sk;
+#pragma unroll
+    for (int r = 0; r < kRuns; ++r)
+      if (grp[r] == k) rs.sc[r] = sk;
+  }
+#pragma unroll
+  for (int r = 0; r < kRuns; ++r) rs.rc[r] = __frcp_rn(rs.sc[r]);
+}
+
+// E4M3 codes of n values x / sc (|x / sc| <= upper_max: div2_bounded).
+template <int N>
+__device__ __forceinline__ void quantize_dyn(float* x, float sc, float rc) {
+#pragma unroll
+  for (int j = 0; j < N / 2; ++j) {
+    const float2 q = div2_bounded(make_float2(x[2 * j], x[2 * j + 1]), make_float2(sc, sc),
+                                  make_float2(rc, rc));
+    x[2 * j] = q.x;
+    x[2 * j + 1] = q.y;
+  }
+}
+
+__device__ __forceinline__ void store_q_head_groups(QHead& v, unsigned char* op, int nope, int l8,
+                                                    const RunScales& rs) {
+#pragma unroll
+  for (int k = 0; k < kMaxChunks; ++k) {
+    const int c = l8 + 8 * k;
+    if (c < nope / 8) {
+      float x[8];
+      unpack8(v.nope[k], x);
+      quantize_dyn<8>(x, rs.sc[k], rs.rc[k]);
+      st_v2(op + 8 * c, pack8_e4m3(x));
+    }
+  }
+  quantize_dyn<4>(v.y, rs.sc[kMaxChunks], rs.rc[kMaxChunks]);
+  quantize_dyn<4>(v.y + 4, rs.sc[kMaxChunks + 1], rs.rc[kMaxChunks + 1]);
+  st_u32(op + nope + 4 * l8, pack4_e4m3(v.y));
+  st_u32(op + nope + kRope / 2 + 4 * l8, pack4_e4m3(v.y + 4));
+}
+
+// Static, per-head and per-group scales: persistent warp tasks
+// [latent rows | row x quad].
 template <int QMODE, int FP8, int STYLE>
 __global__ void __launch_bounds__(kThreads) mla_quant_kernel(const MlaArgs a) {
   extern __shared__ int smem[];
@@ -422,6 +510,13 @@ __global__ void __launch_bounds__(kThreads) mla_quant_kernel(const MlaArgs a) {
     QHead v;
     load_q_head<STYLE>(a.q + static_cast<int64_t>(t) * a.q_tok + static_cast<int64_t>(h) * a.q_head,
                        a.nope, l8, c, s, v);
+    if (QMODE == FQR_MLA_Q_GROUP) {
+      RunScales rs;
+      group_scales(a, v, l8, gmask,
+                   a.q_scale + (static_cast<int64_t>(t) * a.Hq + h) * a.q_ng, rs);
+      store_q_head_groups(v, a.q_out + (static_cast<int64_t>(t) * a.Hq + h) * W, a.nope, l8, rs);
+      continue;
+    }
     float sc = 0.0f, rc = 0.0f;
     if (QMODE == FQR_MLA_Q_HEAD) {
       float mx = q_head_amax(v, a.nope, l8);
@@ -571,6 +666,12 @@ int launch_mla(const fqr_mla_params& p, cudaStream_t stream) {
   a.kv_scale = p.kv_scale; a.flags = p.flags;
   a.q_quant = p.q_quant; a.q_scale_inv = p.q_scale_inv; a.upper_max = p.upper_max;
   a.q_out = static_cast<unsigned char*>(p.q_out); a.q_scale = p.q_scale;
+  a.q_ng = 1;
+  if (p.q_quant == FQR_MLA_Q_GROUP) {
+    const int W = p.nope_dim + p.rope_dim;
+    a.q_ng = (W + p.q_group - 1) / p.q_group;
+    a.gdiv = FastDiv(static_cast<uint32_t>(p.q_group));
+  }
 
   if (p.q_quant == FQR_MLA_Q_TOKEN) {
     MlaKernel k = p.cache_fp8 ? (p.rope_style == 0 ? mla_token_kernel<1, 0> : mla_token_kernel<1, 1>)
@@ -593,7 +694,8 @@ int launch_mla(const fqr_mla_params& p, cudaStream_t stream) {
   }
   if (p.q_quant != FQR_MLA_Q_NONE) {
     MlaKernel k = p.q_quant == FQR_MLA_Q_STATIC ? select_quant<FQR_MLA_Q_STATIC>(p.cache_fp8, p.rope_style)
-                                                : select_quant<FQR_MLA_Q_HEAD>(p.cache_fp8, p.rope_style);
+                  : p.q_quant == FQR_MLA_Q_GROUP ? select_quant<FQR_MLA_Q_GROUP>(p.cache_fp8, p.rope_style)
+                                                 : select_quant<FQR_MLA_Q_HEAD>(p.cache_fp8, p.rope_style);
     const int64_t tasks = static_cast<int64_t>(p.T) * (1 + a.qgroups);
     const size_t smem = static_cast<size_t>(2 * p.B + 1) * sizeof(int);
     return launch_persistent(reinterpret_cast<const void*>(k), tasks, smem, stream,

@@ -307,7 +307,7 @@ class MlaRun:
             self.q_scale = torch.from_numpy(q_scale).to(DEV)
             self.qsi = torch.tensor([w.q_scale_inv], dtype=torch.float32, device=DEV)
             self.qq = dict(q_quant=w.q_quant, q_scale_inv=self.qsi, upper_max=w.upper_max,
-                           q_out=self.q_out, q_scale=self.q_scale)
+                           q_out=self.q_out, q_scale=self.q_scale, q_group=w.q_group)
 
     def launch(self, stream=None):
         fqr.concat_mla_cache(self.q, self.kv_c, self.k_pe, self.cs, self.indptr_d, self.seq_d,

@@ -224,7 +224,10 @@ MLA_BAD = {
     "rope_dim_32": (dict(rope_dim=32, q_head_stride=160, q_token_stride=128 * 160,
                          k_pe_stride=32), 2),
     "rank_not_multiple_of_8": (dict(kv_lora_rank=500, kv_c_stride=500), 2),
-    "q_quant_4": (dict(q_quant=4, q_out=FAKE), 1),
+    "q_quant_5": (dict(q_quant=5, q_out=FAKE, q_scale=FAKE), 1),
+    "q_group_zero": (dict(q_quant=4, q_out=FAKE, q_scale=FAKE, q_group=0), 1),
+    "q_group_not_multiple_of_8": (dict(q_quant=4, q_out=FAKE, q_scale=FAKE, q_group=60), 1),
+    "q_group_without_q_scale": (dict(q_quant=4, q_out=FAKE, q_group=64), 1),
     "q_static_without_scale": (dict(q_quant=1, q_out=FAKE), 1),
     "q_dynamic_without_q_scale": (dict(q_quant=2, q_out=FAKE), 1),
     "q_dynamic_upper_max_zero": (dict(q_quant=3, q_out=FAKE, q_scale=FAKE, upper_max=0.0), 1),

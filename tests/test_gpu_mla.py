@@ -1,7 +1,8 @@
 """GPU parity of fqr_concat_mla_cache against the oracle, through the C ABI:
 the full-size MLA decode workload, BF16 and NeoX variants, ragged prefill
 with empty requests, malformed metadata, and Q quantised to FP8 (static,
-per token, per head; bitwise codes and scales)."""
+per token, per head, per group of a head's values; bitwise codes and
+scales)."""
 import numpy as np
 import pytest
 import torch
@@ -79,6 +80,34 @@ def test_mla_decode_q_fp8_parity(q_quant):
     run(workloads.mla_decode(q_quant=q_quant))
 
 
+@pytest.mark.parametrize("group", [64, 128])
+def test_mla_decode_q_fp8_group_parity(group):
+    """The full-size MLA decode with per-group Q scales: 3 groups of 64 per
+    192-wide head, or 2 (the 128 nope values and the 64 rope values)."""
+    run(workloads.mla_decode(q_quant=4, q_group=group))
+
+
+@pytest.mark.parametrize("group", [8, 16, 24, 64, 96, 128, 192, 256])
+@pytest.mark.parametrize("style", [1, 0])
+def test_mla_q_fp8_group_ragged(group, style):
+    """Ragged batches, empty requests, an all-zero token and an all-zero group
+    (floor scales), nope 64 or 128, every group size class: groups inside a
+    lane's run, across the nope / rope boundary, longer than the head."""
+    rng = np.random.default_rng(group * 2 + style)
+    B = 6
+    n = rng.integers(0, 25, B)
+    n[1] = 0
+    L = rng.integers(0, 90, B) + n
+    nope = 64 if group % 16 else 128
+    w = workloads.make_mla(seed=80 + group + style, n_new=n, seq_lens=L, Hq=19, block_size=16,
+                           max_blocks=int(np.ceil(L.max() / 16)) + 1, rope_style=style,
+                           nope_dim=nope, kv_lora_rank=128, cos_sin_rows=int(L.max()) + 1,
+                           q_quant=4, q_group=group, upper_max=240.0 if style else 448.0)
+    w.q[0] = 0                                  # an all-zero token
+    w.q[1, 3, :16] = 0                          # a zero run at the start of a head
+    run(w)
+
+
 @pytest.mark.parametrize("q_quant", [1, 2, 3])
 @pytest.mark.parametrize("style", [1, 0])
 @pytest.mark.parametrize("upper", [448.0, 240.0])
@@ -114,7 +143,7 @@ def test_mla_q_fp8_per_token_wide_rows_many_clusters(style):
     run(w)
 
 
-@pytest.mark.parametrize("q_quant", [1, 2, 3])
+@pytest.mark.parametrize("q_quant", [1, 2, 3, 4])
 def test_mla_q_fp8_with_bf16_latent(q_quant):
     """FP8 Q with a BF16 latent cache (every kernel variant's FP8 = 0 side)."""
     rng = np.random.default_rng(60 + q_quant)
@@ -123,7 +152,7 @@ def test_mla_q_fp8_with_bf16_latent(q_quant):
     w = workloads.make_mla(seed=61 + q_quant, n_new=n, seq_lens=L, Hq=20, block_size=32,
                            max_blocks=int(np.ceil(L.max() / 32)) + 1, kv_lora_rank=128,
                            cos_sin_rows=int(L.max()) + 1, cache_fp8=0, q_quant=q_quant,
-                           q_scale_inv=25.0)
+                           q_scale_inv=25.0, q_group=64)
     run(w)
 
 
@@ -140,10 +169,52 @@ def test_mla_q_fp8_per_token_few_heads(Hq):
     run(w)
 
 
-@pytest.mark.parametrize("q_quant", [1, 2, 3])
+@pytest.mark.parametrize("q_quant", [1, 2, 3, 4])
 def test_mla_q_fp8_malformed_writes_nothing(q_quant):
     w = workloads.make_mla(seed=4, n_new=[2, 1, 1], seq_lens=[4, 3, 2], Hq=8, block_size=4,
-                           max_blocks=2, kv_lora_rank=64, cos_sin_rows=8, q_quant=q_quant)
+                           max_blocks=2, kv_lora_rank=64, cos_sin_rows=8, q_quant=q_quant,
+                           q_group=32)
     r, rep = run(w, q_indptr=np.array([0, 3, 2, 4], np.int32))
     assert rep == {"flagged": True}
     assert torch.equal(r.q_out, r.q_out_before)
+
+
+@pytest.mark.parametrize("graph", [False, True])
+def test_back_to_back_launches_read_each_others_writes(graph):
+    """Two fqr_concat_mla_cache launches on one stream with nothing in between
+    (each launch lets the next start its prologue early: programmatic
+    dependent launch, also inside a CUDA graph).  The second reads the q the
+    first rotated in place, so q ends up rotated twice: exactly the oracle
+    applied twice.  A launch that read q before the preceding launch had
+    finished would leave it rotated once."""
+    import oracle
+    from tests.gpu_harness import _np
+    rng = np.random.default_rng(90)
+    n = rng.integers(1, 4, 24)
+    L = rng.integers(1, 3000, 24) + n
+    w = workloads.make_mla(seed=91, n_new=n, seq_lens=L, Hq=128, block_size=64,
+                           max_blocks=int(np.ceil(L.max() / 64)) + 1, kv_lora_rank=512,
+                           cos_sin_rows=int(L.max()) + 1)
+    r = MlaRun(w)
+    lat0 = _np(r.latent).copy()
+    if graph:
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            r.launch(stream=s)
+            r.launch(stream=s)
+        g.replay()
+    else:
+        r.launch()
+        r.launch()
+    torch.cuda.synchronize()
+    q, lat, fl = w.q.copy(), lat0.copy(), np.zeros(w.B, np.int32)
+    for _ in range(2):
+        assert oracle.concat_mla_cache(w, q, lat, fl) == 0
+    assert np.array_equal(_np(r.q), q)
+    assert np.array_equal(_np(r.latent), lat)
+    assert not r.flags.cpu().numpy().any()
+    assert not np.array_equal(q, w.q)
+    if graph:
+        del g
