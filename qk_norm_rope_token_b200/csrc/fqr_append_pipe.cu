@@ -4,7 +4,7 @@
 // Method: FlashInfer PR #5956, section "Contract" (see fqr_head.cuh for the
 // per-head arithmetic).
 //
-// One block = 1 producer warp + 8 consumer warps; persistent grid, every
+// One block = 1 producer warp + 7 consumer warps; persistent grid, every
 // block resident; each block owns a contiguous range of units (a unit is one
 // packed row, or a chunk of its heads for very wide rows).
 //   * the producer streams each unit into a ring of shared-memory stages with
@@ -18,7 +18,7 @@
 //   * consumer warps take 4 heads at a time from the stage (fqr_head.cuh),
 //     store straight to out_q / the cache slot and release the stage on its
 //     "empty" mbarrier; the quad -> warp assignment rotates every unit.
-//   * the 8 consumer warps split the last-page tail of a request's last row
+//   * the consumer warps split the last-page tail of a request's last row
 //     evenly between them (after releasing the stage); consumer warps of the
 //     grid zero the tails of requests that append nothing.
 //   * every block validates the whole batch first; every wait is bounded
@@ -28,7 +28,7 @@
 
 namespace fqr {
 
-constexpr int kConsumers = 8;
+constexpr int kConsumers = 7;
 constexpr int kPipeThreads = (kConsumers + 1) * 32;
 constexpr int kMaxStages = 8;
 constexpr int kFixedSmem = 1280;  // barriers (128) + fp32 weights (1024) + spare
@@ -241,7 +241,7 @@ __device__ void consume(const PipeArgs& a, const unsigned char* stages, uint64_t
       s = 0;
       ph ^= 1u;
     }
-    rot = (rot + nq) & (kConsumers - 1);
+    rot = (rot + nq) % kConsumers;
     if (++c == a.nchunks) {
       c = 0;
       ++t;
@@ -263,8 +263,11 @@ __device__ void zero_empty_request_tails(const PipeArgs& a, const int* s_indptr,
   }
 }
 
-// Two resident blocks per SM: 18 warps, at most 5 on each of the 4 sub-partition
-// register files (16K registers each), so at most 96 registers a thread.
+// Two resident blocks per SM: 16 warps, 4 on each of the 4 sub-partition
+// register files (16K registers each), so up to 128 registers a thread.
+// (Eight consumer warps a block would put 5 warps on some sub-partitions and
+// cap a thread at 96 registers: measured slower, 86.1 -> 79.5 us per launch of
+// the ragged FP8 prefill with seven.)
 template <int POLICY, int STYLE>
 __global__ void __launch_bounds__(kPipeThreads, 2) pipe_append_kernel(const PipeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];

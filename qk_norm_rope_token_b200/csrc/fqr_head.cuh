@@ -376,20 +376,141 @@ __device__ __forceinline__ int quad_kind(const HeadParams& a, int h0) {
 // summation order (four lane chains, then the group's xor tree) can change
 // it.  One rounding to fp32, then +eps, the square root and the reciprocal,
 // each correctly rounded (rn_recip_sqrt).
-__device__ __forceinline__ float inv_rms(const float2* y, float eps, unsigned gmask) {
-  double s[4] = {0.0, 0.0, 0.0, 0.0};
+//
+// The squares are formed in binary64 from two conversions, to balance the
+// pipes: the first value of each pair by the hardware conversion, the second
+// by integer operations on its fp32 bits u -- for a BF16 value (8 significant
+// bits) the binary64 high word is ((u >> 3) & 0x0FFFFFFF) + ((1023 - 127) << 20)
+// with a zero low word (the sign is dropped: only the square is used).  That
+// is exact for every finite nonzero normal value; a zero or subnormal becomes
+// a value below 2^-126, whose square cannot reach the fp32 rounding of any
+// mean square that does not itself round to zero; an Inf becomes 2^128, as
+// good as infinite here (the mean square overflows, 1/sqrt gives 0); only a
+// NaN would turn finite, so when the mean square overflows, the head's values
+// are checked for a NaN (a rare branch), which then makes the result NaN.
+template <int N>
+__device__ __forceinline__ void inv_rms_n(float2 (*y)[8], float eps, unsigned gmask, float* inv) {
+  double ss[N];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const double u = y[j].x, v = y[j].y;
-    s[(j & 1) * 2] = fma(u, u, s[(j & 1) * 2]);
-    s[(j & 1) * 2 + 1] = fma(v, v, s[(j & 1) * 2 + 1]);
+  for (int n = 0; n < N; ++n) {
+    double s[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t uy = __float_as_uint(y[n][j].y);
+      const double u = y[n][j].x;
+      const double v =
+          __hiloint2double(static_cast<int>(__umulhi(uy & 0x7FFF0000u, 1u << 29) + 0x38000000u), 0);
+      s[(j & 1) * 2] = fma(u, u, s[(j & 1) * 2]);
+      s[(j & 1) * 2 + 1] = fma(v, v, s[(j & 1) * 2 + 1]);
+    }
+    ss[n] = (s[0] + s[1]) + (s[2] + s[3]);
   }
-  double ss = (s[0] + s[1]) + (s[2] + s[3]);
-  ss += __shfl_xor_sync(gmask, ss, 4);
-  ss += __shfl_xor_sync(gmask, ss, 2);
-  ss += __shfl_xor_sync(gmask, ss, 1);
-  const float ms = __double2float_rn(ss * (1.0 / kHeadDim));
-  return rn_recip_sqrt(__fadd_rn(ms, eps));
+#pragma unroll
+  for (int m = 4; m >= 1; m >>= 1) {
+#pragma unroll
+    for (int n = 0; n < N; ++n) ss[n] += __shfl_xor_sync(gmask, ss[n], m);
+  }
+#pragma unroll
+  for (int n = 0; n < N; ++n) {
+    float ms = __double2float_rn(ss[n] * (1.0 / kHeadDim));
+    if (__builtin_expect(ms == INFINITY, 0)) {  // the whole 8-lane group agrees on ms
+      bool nan = false;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) nan |= isnan(y[n][j].x) || isnan(y[n][j].y);
+      if (__any_sync(gmask, nan)) ms = __int_as_float(0x7FC00000);
+    }
+    inv[n] = rn_recip_sqrt(__fadd_rn(ms, eps));
+  }
+}
+__device__ __forceinline__ float inv_rms(float2* y, float eps, unsigned gmask) {
+  float inv;
+  inv_rms_n<1>(reinterpret_cast<float2(*)[8]>(y), eps, gmask, &inv);
+  return inv;
+}
+
+// The RoPE of one head's lane slices y with the lane's cos/sin values c, s
+// (NeoX: pairs (i, i + 64) across the two chunks; GPT-J: pairs (2i, 2i + 1)
+// inside a float2, dims >= rot passing through).
+template <int STYLE>
+__device__ __forceinline__ void rope_head(float2* y, const float2* c, const float2* s, int rot,
+                                          int l8) {
+  if (STYLE == 0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) rotate_pairs2(y[j], y[4 + j], c[j], s[j]);
+  } else {  // dims >= rot_dim pass through untouched
+    const int half = rot >> 1;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (4 * l8 + j < half) rotate_pair(y[j].x, y[j].y, c[j].x, s[j].x);
+      if (32 + 4 * l8 + j < half) rotate_pair(y[4 + j].x, y[4 + j].y, c[j].y, s[j].y);
+    }
+  }
+}
+
+// Quantisation and store of a normed and rotated Q head (out_q) or K head (its
+// KV slot, or row r of the caller-owned K output).
+template <int POLICY, int KIND>
+__device__ __forceinline__ void output_qk_head(const HeadParams& a, const RowCtx& r, int h,
+                                               float2* y, int l8, unsigned gmask) {
+  constexpr int ES = POLICY == 0 ? 2 : 1;
+  if (KIND == kQHead) {
+    char* dst = static_cast<char*>(a.out_q) +
+                (static_cast<int64_t>(r.t) * a.Hq + h) * kHeadDim * ES;
+    if (POLICY == 1) {
+      float amax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fmaxf(fabsf(y[j].x), fabsf(y[j].y)));
+      amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 4));
+      amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 2));
+      amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 1));
+      const float qs = __fdiv_rn(fmaxf(amax, 1e-6f), a.upper_max);
+      if (l8 == 0) a.q_scale[r.qs + static_cast<int64_t>(h) * (a.qs_prefill ? a.qs_ld : 1)] = qs;
+      const float rq = __frcp_rn(qs);
+      const float2 b2 = make_float2(qs, qs), r2 = make_float2(rq, rq);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[j] = div2_bounded(y[j], b2, r2);
+    } else if (POLICY == 2) {
+      const float qsi = __ldg(a.q_scale_inv);
+      const float2 qv = make_float2(qsi, qsi);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[j] = mul2(y[j], qv);
+    }
+    store_head<POLICY>(dst, y, l8);
+  } else {
+    const int kh = h - a.Hq;
+    char* page_base = a.k_cache + static_cast<int64_t>(r.page) * a.k_page_bytes;
+    char* dst = a.out_k != nullptr
+                    ? a.out_k + (static_cast<int64_t>(r.t) * a.Hkv + kh) * kHeadDim * ES
+                    : page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
+    if (POLICY != 0) divide_pairs(y, __ldg(a.k_scale));
+    store_head<POLICY>(dst, y, l8);
+  }
+}
+
+// Norm + RoPE + output of N heads h[0..N) of one kind (KIND: kQHead or
+// kKHead) of row r at once, from their lane slices y (unpacked): the heads'
+// dependency chains interleave, and they share the cos/sin values and the
+// norm weights.
+template <int POLICY, int STYLE, int KIND, int N, class W>
+__device__ __forceinline__ void process_qk_heads(const HeadParams& a, const RowCtx& r, const int* h,
+                                                 float2 (*y)[8], const float2* c, const float2* s,
+                                                 const W& wts, int l8, unsigned gmask) {
+  if (KIND == kQHead ? a.has_qw : a.has_kw) {
+    float inv[N];
+    inv_rms_n<N>(y, a.eps, gmask, inv);
+    float2 w[8];
+    load_weights(wts, KIND == kQHead, l8, w);
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+      const float2 iv = make_float2(inv[n], inv[n]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[n][j] = mul2(mul2(y[n][j], iv), w[j]);
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < N; ++n) rope_head<STYLE>(y[n], c, s, a.rot, l8);
+#pragma unroll
+  for (int n = 0; n < N; ++n) output_qk_head<POLICY, KIND>(a, r, h[n], y[n], l8, gmask);
 }
 
 // Norm + RoPE + quantisation + store of head h of row r.  xa/xb: the lane's two
@@ -424,63 +545,14 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
     return;
   }
 
+  float2 yy[1][8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) yy[0][j] = y[j];
   const bool is_q = KIND == kQHead || (KIND == kAnyHead && h < a.Hq);
-  // -------------------------------------------------------------- RMSNorm
-  if (is_q ? a.has_qw : a.has_kw) {
-    const float inv = inv_rms(y, a.eps, gmask);
-    const float2 iv = make_float2(inv, inv);
-    float2 w[8];
-    load_weights(wts, is_q, l8, w);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = mul2(mul2(y[j], iv), w[j]);
-  }
-
-  // ----------------------------------------------------------------- RoPE
-  if (STYLE == 0) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) rotate_pairs2(y[j], y[4 + j], c[j], s[j]);
-  } else {  // dims >= rot_dim pass through untouched
-    const int half = a.rot >> 1;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (4 * l8 + j < half) rotate_pair(y[j].x, y[j].y, c[j].x, s[j].x);
-      if (32 + 4 * l8 + j < half) rotate_pair(y[4 + j].x, y[4 + j].y, c[j].y, s[j].y);
-    }
-  }
-
-  // --------------------------------------------------------------- output
-  if (is_q) {
-    char* dst = static_cast<char*>(a.out_q) +
-                (static_cast<int64_t>(r.t) * a.Hq + h) * kHeadDim * ES;
-    if (POLICY == 1) {
-      float amax = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fmaxf(fabsf(y[j].x), fabsf(y[j].y)));
-      amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 4));
-      amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 2));
-      amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 1));
-      const float qs = __fdiv_rn(fmaxf(amax, 1e-6f), a.upper_max);
-      if (l8 == 0) a.q_scale[r.qs + static_cast<int64_t>(h) * (a.qs_prefill ? a.qs_ld : 1)] = qs;
-      const float rq = __frcp_rn(qs);
-      const float2 b2 = make_float2(qs, qs), r2 = make_float2(rq, rq);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) y[j] = div2_bounded(y[j], b2, r2);
-    } else if (POLICY == 2) {
-      const float qsi = __ldg(a.q_scale_inv);
-      const float2 qv = make_float2(qsi, qsi);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) y[j] = mul2(y[j], qv);
-    }
-    store_head<POLICY>(dst, y, l8);
-  } else {  // ------------------------------------------------------------ K
-    const int kh = h - a.Hq;
-    char* page_base = a.k_cache + static_cast<int64_t>(r.page) * a.k_page_bytes;
-    char* dst = a.out_k != nullptr
-                    ? a.out_k + (static_cast<int64_t>(r.t) * a.Hkv + kh) * kHeadDim * ES
-                    : page_base + r.slot_row * a.row_bytes + kh * kHeadDim * ES;
-    if (POLICY != 0) divide_pairs(y, __ldg(a.k_scale));
-    store_head<POLICY>(dst, y, l8);
-  }
+  if (is_q)
+    process_qk_heads<POLICY, STYLE, kQHead, 1>(a, r, &h, yy, c, s, wts, l8, gmask);
+  else
+    process_qk_heads<POLICY, STYLE, kKHead, 1>(a, r, &h, yy, c, s, wts, l8, gmask);
 }
 
 // As process_head_cs, loading the cos/sin values from cs_row first (V heads

@@ -84,9 +84,9 @@ def test_describe_plan_names_the_schedule_and_variants():
     assert "1664 warp tasks" in d and "warp-level batch check" in d and "bulk" not in d
     d = bench.describe_plan(dict(lat, warp_check=0, bulk_tails=1, request_tails=1))
     assert "block batch prologue" in d and "bulk-copy tails" in d and "own the tails" in d
-    d = bench.describe_plan(dict(schedule=2, grid=296, block_threads=288, tasks=9212,
+    d = bench.describe_plan(dict(schedule=2, grid=296, block_threads=256, tasks=9212,
                                  warp_check=0, bulk_tails=0, request_tails=0))
-    assert "streaming schedule" in d and "296 blocks of 288 threads" in d and "9212 units" in d
+    assert "streaming schedule" in d and "296 blocks of 256 threads" in d and "9212 units" in d
 
 
 def test_prefill_replicas_keep_the_batch_shape():

@@ -174,7 +174,7 @@ PLANS = {
     "fp8_decode_dynamic": dict(schedule=1, block_threads=256, tasks=5376, warp_check=0,
                                bulk_tails=1, request_tails=0),
     "decode_out_kv_bf16": dict(schedule=1, block_threads=384, warp_check=1),
-    "ragged_prefill_fp8": dict(schedule=2, block_threads=288, warp_check=0),
+    "ragged_prefill_fp8": dict(schedule=2, block_threads=256, grid=296, warp_check=0),
 }
 
 
@@ -313,3 +313,51 @@ def test_cuda_graph_capture_and_replay_is_bitwise_eager(schedule):
             assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
     del g
     r.check()
+
+
+def _special_heads(w, seed):
+    """Plant special values into the Q and K heads of w's rows (in place):
+    every case lands in a Q head and in a K head of some row."""
+    rng = np.random.default_rng(seed)
+    D = 128
+
+    def put(r, h, fn):
+        head = w.qkv[r, h * D:(h + 1) * D]
+        fn(head, rng)
+
+    cases = [
+        lambda x, g: x.__setitem__(5, 0x7FC0),                     # NaN, odd slot
+        lambda x, g: x.__setitem__(6, 0xFFC1),                     # NaN, even slot
+        lambda x, g: x.__setitem__(3, 0x7F80),                     # +Inf
+        lambda x, g: x.__setitem__(100, 0xFF80),                   # -Inf
+        lambda x, g: x.__setitem__(slice(None), g.choice([0x7F7F, 0xFF7F, 0x7F70], D)),  # ~BF16 max
+        lambda x, g: x.__setitem__(slice(None), g.integers(1, 0x80, D)),                  # subnormals
+        lambda x, g: x.__setitem__(slice(None), 0),                                      # zeros
+        lambda x, g: (x.__setitem__(slice(None), 0), x.__setitem__(77, 0x3F80)),          # one-hot
+        lambda x, g: x.__setitem__(slice(None), np.where(g.random(D) < 0.5, 0x7149, 0x0DA2)),  # 1e30 / 1e-30
+        lambda x, g: x.__setitem__(slice(None), x & 0x80FF | 0x0080),  # tiny normals
+    ]
+    heads = list(range(w.Hq)) + list(range(w.Hq, w.Hq + w.Hkv))
+    r = 0
+    for i, fn in enumerate(cases):
+        for h in (heads[i % w.Hq], w.Hq + i % w.Hkv):
+            put(r % w.T, h, fn)
+            r += 1
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
+@pytest.mark.parametrize("policy", [0, 1])
+def test_special_values_in_normed_heads(policy, schedule):
+    """Q/K heads holding NaN (at either conversion slot of a pair), +-Inf,
+    values near the BF16 maximum (the mean square overflows), subnormals,
+    zeros, a one-hot head, 1e30 beside 1e-30, and tiny normals, against the
+    oracle: a NaN makes the whole head NaN, an overflowing mean square gives
+    1/sqrt = 0, and everything else matches within the bar."""
+    n = [5, 3, 6, 4]
+    L = [9, 20, 31, 70]
+    w = workloads.make_append(seed=77, n_new=n, seq_lens=L, Hq=16, Hkv=4, page_size=16,
+                              max_pages=6, quant_policy=policy, qkv_sigma=1.0,
+                              cos_sin_rows=128, k_scale=0.05, v_scale=0.05)
+    _special_heads(w, 5)
+    _, rep = run_and_check(w, schedule=schedule)
+    assert not rep.get("flagged")
