@@ -23,8 +23,9 @@ device->host copies of out_q and flags inside the timed region);
 `cpu_baseline` = the CPU oracle on a bounded sample, single-threaded
 (`cpu_baseline_all_cores`: one process per host core on disjoint requests);
 `per_config` (last, compact) adds every named workload measured the same way
-outside the timed region: microseconds per launch, fraction of the peak, and
-the two schedules forced.
+outside the timed region: microseconds per launch, fraction of the peak, the
+two schedules forced, and the floor -- a plain copy kernel moving the same
+bytes in one launch (libfqr_floor.so).
 
 --impl reference times the CPU oracle (the reference arm of this build) on
 the host cores on the same workload, metric and unit.
@@ -138,10 +139,12 @@ def profiled_traffic(workload: str):
     committed ncu record profiles/traffic.json, if it was captured on the
     current append-kernel sources.  Returns (traffic bytes or None, details).
 
-    traffic = dram__bytes_read.sum + 32 x lts__t_sectors_op_write.sum: reads
-    counted at DRAM, writes where they enter L2 (a write-back cache: a
-    launch's last writes are still in L2 when it ends, so dram__bytes_write
-    undercounts them; every sector written reaches DRAM once)."""
+    traffic = dram__bytes_read.sum + 32 x lts__t_sectors_srcnode_gpc_op_write.sum:
+    reads counted at DRAM, writes where the SMs issue them into L2 (a
+    write-back cache: a launch's last writes are still in L2 when it ends, so
+    dram__bytes_write undercounts them; every sector written reaches DRAM
+    once).  lts__t_sectors_op_write.sum would count again the writes that
+    cross the die-to-die fabric to their home L2 slice."""
     try:
         with open(TRAFFIC_RECORD) as f:
             rec = json.load(f)
@@ -152,10 +155,11 @@ def profiled_traffic(workload: str):
     e = rec.get("workloads", {}).get(workload)
     if not e:
         return None, {"note": f"no traffic record for {workload}"}
-    t = int(e["dram_read_bytes"]) + int(e["l2_write_bytes"])
-    return t, {"dram_read": int(e["dram_read_bytes"]), "l2_write": int(e["l2_write_bytes"]),
+    t = int(e["dram_read_bytes"]) + int(e["gpc_write_bytes"])
+    return t, {"dram_read": int(e["dram_read_bytes"]), "sm_write_into_l2": int(e["gpc_write_bytes"]),
                "dram_write": int(e["dram_write_bytes"]),
-               "basis": "ncu: dram__bytes_read.sum + 32 x lts__t_sectors_op_write.sum per launch"}
+               "basis": "ncu: dram__bytes_read.sum + 32 x lts__t_sectors_srcnode_gpc_op_write.sum "
+                        "per launch (profiles/traffic.json)"}
 
 
 class ClockSampler:
@@ -377,6 +381,41 @@ class MlaBench:
         rc = self.fqr.concat_mla_cache_raw(self.params[i % self.R], stream_handle)
         if rc != 0:
             raise self.fqr.FqrError(rc)
+
+
+class FloorBench:
+    """The plain copy kernel of libfqr_floor.so moving a workload's read and
+    write bytes (workloads.append_bytes) in one launch, over replicas of its
+    source and destination buffers (a cycle larger than L2), launched like
+    the fused kernel (programmatic dependent launch).  Its time per launch is
+    the floor the fused kernel is compared with on small workloads."""
+
+    def __init__(self, torch, device, read_bytes, write_bytes, min_bytes=3 * L2_BYTES,
+                 max_replicas=64):
+        import ctypes
+        path = os.path.join(ROOT, "qk_norm_rope_token_b200", "libfqr_floor.so")
+        self.lib = ctypes.CDLL(path)
+        self.lib.fqr_floor_copy.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint64,
+                                            ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p]
+        self.lib.fqr_floor_copy.restype = ctypes.c_int
+        self.rb = -(-int(read_bytes) // 16) * 16
+        self.wb = -(-int(write_bytes) // 16) * 16
+        per = self.rb + self.wb
+        self.R = int(min(max_replicas, max(2, math.ceil(min_bytes / per))))
+        self.src = [torch.randint(0, 1 << 30, (max(4, self.rb // 4),), dtype=torch.int32,
+                                  device=device) for _ in range(self.R)]
+        self.dst = [torch.empty(max(4, self.wb // 4), dtype=torch.int32, device=device)
+                    for _ in range(self.R)]
+        self.bytes = [per] * self.R
+        vec = max(self.rb, self.wb) // 16
+        self.blocks = int(min(4 * 148, max(1, -(-vec // 256))))
+
+    def launch(self, i, stream_handle):
+        k = i % self.R
+        rc = self.lib.fqr_floor_copy(self.src[k].data_ptr(), self.dst[k].data_ptr(), self.rb,
+                                     self.wb, self.blocks, stream_handle)
+        if rc != 0:
+            raise RuntimeError(f"fqr_floor_copy failed: {rc}")
 
 
 def time_launches(torch, bench, steps, warmup, repeats=1, graph_chunk=1000, barrier=None,
@@ -768,8 +807,10 @@ def measure_per_config(torch, fqr, dev, peak, warmup=50, repeats=3):
     """Every named workload, timed like the headline (median of `repeats`
     regions), in a compact form: us = microseconds per launch (automatic
     schedule), frac = algorithmic bytes / time / peak, lat / str = us per
-    launch with the latency / streaming schedule forced, MB = algorithmic
-    megabytes per launch, T = tokens per launch."""
+    launch with the latency / streaming schedule forced, floor = us per
+    launch of a plain copy kernel moving the same read and write bytes
+    (FloorBench), MB = algorithmic megabytes per launch, T = tokens per
+    launch."""
     out = {}
 
     def timed(b):
@@ -787,8 +828,13 @@ def measure_per_config(torch, fqr, dev, peak, warmup=50, repeats=3):
             for st in b.reps:
                 st["params"].schedule = sched
             e[label] = _short(timed(b)[0])
-        out[name] = e
+        nb = workloads.append_bytes(b.ws[0])
         del b
+        torch.cuda.empty_cache()
+        f = FloorBench(torch, dev, nb["read"], nb["write"])
+        e["floor"] = _short(timed(f)[0])     # the plain copy of the same bytes
+        out[name] = e
+        del f
         torch.cuda.empty_cache()
     for name in workloads.MLA_CONFIGS:
         m = MlaBench(torch, fqr, dev, name=name)

@@ -42,7 +42,23 @@ def _stale() -> bool:
     return os.path.getmtime(LIB) < max(os.path.getmtime(f) for f in inputs)
 
 
+FLOOR_SRC = os.path.join(CSRC, "copy_floor.cu")
+FLOOR_LIB = os.path.join(PKG, "libfqr_floor.so")
+
+
+def build_floor(force: bool = False) -> str:
+    """libfqr_floor.so: the bench's plain copy kernel (not part of libfqr)."""
+    if (not force and os.path.exists(FLOOR_LIB)
+            and os.path.getmtime(FLOOR_LIB) >= os.path.getmtime(FLOOR_SRC)):
+        return FLOOR_LIB
+    tmp = FLOOR_LIB + ".tmp%d" % os.getpid()
+    subprocess.run([nvcc(), *NVCC_FLAGS, "-shared", FLOOR_SRC, "-o", tmp], check=True)
+    os.replace(tmp, FLOOR_LIB)
+    return FLOOR_LIB
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    build_floor(force)
     if not force and not _stale():
         return LIB
     flags = list(NVCC_FLAGS)

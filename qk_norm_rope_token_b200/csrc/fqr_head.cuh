@@ -545,14 +545,16 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
     return;
   }
 
-  float2 yy[1][8];
+  if constexpr (KIND != kVHead) {
+    float2 yy[1][8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) yy[0][j] = y[j];
-  const bool is_q = KIND == kQHead || (KIND == kAnyHead && h < a.Hq);
-  if (is_q)
-    process_qk_heads<POLICY, STYLE, kQHead, 1>(a, r, &h, yy, c, s, wts, l8, gmask);
-  else
-    process_qk_heads<POLICY, STYLE, kKHead, 1>(a, r, &h, yy, c, s, wts, l8, gmask);
+    for (int j = 0; j < 8; ++j) yy[0][j] = y[j];
+    const bool is_q = KIND == kQHead || (KIND == kAnyHead && h < a.Hq);
+    if (is_q)
+      process_qk_heads<POLICY, STYLE, kQHead, 1>(a, r, &h, yy, c, s, wts, l8, gmask);
+    else
+      process_qk_heads<POLICY, STYLE, kKHead, 1>(a, r, &h, yy, c, s, wts, l8, gmask);
+  }
 }
 
 // As process_head_cs, loading the cos/sin values from cs_row first (V heads

@@ -267,3 +267,19 @@ def test_pipeline_rejects_bad_arguments_before_any_cuda_call(fqr):
     assert L.fqr_pipeline_submit(None, FAKE, FAKE) == fqr.FQR_EINVAL
     assert L.fqr_pipeline_join(None, None) == fqr.FQR_EINVAL
     assert L.fqr_pipeline_fork(None, None) == fqr.FQR_EINVAL
+
+
+def test_floor_copy_library_loads_and_checks_arguments():
+    """libfqr_floor.so (the bench's plain copy kernel) exports fqr_floor_copy
+    and rejects invalid arguments before any CUDA call."""
+    import ctypes
+    path = os.path.join(ROOT, "qk_norm_rope_token_b200", "libfqr_floor.so")
+    lib = ctypes.CDLL(path)
+    f = lib.fqr_floor_copy
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint64,
+                  ctypes.c_int, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    assert f(FAKE, FAKE, 24, 32, 4, None) == 1          # size not a multiple of 16
+    assert f(FAKE + 8, FAKE, 32, 32, 4, None) == 1      # misaligned source
+    assert f(None, FAKE, 32, 32, 4, None) == 1          # no source
+    assert f(FAKE, FAKE, 32, 32, 0, None) == 1          # no blocks

@@ -120,7 +120,7 @@ def test_traffic_record_needs_the_current_kernel_sources(tmp_path, monkeypatch):
     sys.path.insert(0, ROOT)
     import bench
     rec = {"kernel_sources": bench.kernel_source_hash(),
-           "workloads": {"ragged_prefill_fp8": {"dram_read_bytes": 100, "l2_write_bytes": 50,
+           "workloads": {"ragged_prefill_fp8": {"dram_read_bytes": 100, "gpc_write_bytes": 50,
                                                 "dram_write_bytes": 40}}}
     path = tmp_path / "traffic.json"
     path.write_text(json.dumps(rec))
