@@ -243,8 +243,7 @@ def replica_workloads(name, min_bytes=3 * L2_BYTES, max_replicas=64, seed_offset
         def make(seed=None, _f=workloads.APPEND_CONFIGS[name], **kw):
             return workloads.shrink_cache(_f(**kw) if seed is None else _f(seed=seed, **kw))
     base = make()
-    per = workloads.append_bytes(base)["total"]
-    R = int(min(max_replicas, max(2, math.ceil(min_bytes / per))))
+    R = replica_count(base, min_bytes, max_replicas)
     base_n = np.diff(base.q_indptr)
     ws = []
     for r in range(R):
@@ -643,7 +642,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic", "config": config_block(w, None),
+        "data": "synthetic", "config": config_block(w),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": len(jobs), "kind": "oracle",
                          "sample": f"{len(jobs)} processes x {args.steps} steps, each step one "
                                    f"call over {tokens} request(s) of the process's own share of "
@@ -678,19 +677,25 @@ def max_over_ranks(torch, dist, x: float, device) -> float:
     return float(t.item())
 
 
-def config_block(w, bench):
-    c = {"workload": w.name, "tokens_per_step": w.T, "requests": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
-         "head_dim": 128, "page_size": w.page_size, "quant_policy": w.quant_policy,
-         "io_dtype": "bf16 in, " + ("bf16" if w.quant_policy == 0 else "e4m3") + " out",
-         "parallelism": "replicas"}
-    if bench is not None:
-        seeds = sorted({x.seed for x in bench.ws})
-        c["replicas"] = bench.R
-        c["seeds"] = (f"{seeds[0]} (+7919 per replica): workload draws; the replicas keep the "
-                      f"first one's token counts" if len(seeds) > 1 else str(seeds[0]))
-        c["l2"] = (f"inputs larger than L2: each step uses its own replica of the step inputs "
-                   f"({bench.R} replicas, {sum(bench.bytes) / 1e6:.0f} MB rotated per cycle)")
-    return c
+def replica_count(w, min_bytes=3 * L2_BYTES, max_replicas=64) -> int:
+    """Replicas a bench of workload w rotates over (replica_workloads)."""
+    per = workloads.append_bytes(w)["total"]
+    return int(min(max_replicas, max(2, math.ceil(min_bytes / per))))
+
+
+def config_block(w):
+    """The workload of a line, identical for both arms: its shape, and how the
+    GPU arm keeps the timed steps' inputs out of L2 (derived from w alone)."""
+    R = replica_count(w)
+    per = workloads.append_bytes(w)["total"]
+    return {"workload": w.name, "tokens_per_step": w.T, "requests": w.B, "Hq": w.Hq,
+            "Hkv": w.Hkv, "head_dim": 128, "page_size": w.page_size,
+            "quant_policy": w.quant_policy,
+            "io_dtype": "bf16 in, " + ("bf16" if w.quant_policy == 0 else "e4m3") + " out",
+            "parallelism": "replicas", "replicas": R,
+            "seeds": f"{w.seed} (+7919 per replica); the replicas keep the first draw's token counts",
+            "l2": (f"inputs larger than L2: each step uses its own replica of the step inputs "
+                   f"({R} replicas, about {R * per / 1e6:.0f} MB rotated per cycle)")}
 
 
 # --------------------------------------------------------------------- main
@@ -761,7 +766,7 @@ def main(argv=None):
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "gpu_launches": args.steps,
-        "config": config_block(bench.ws[0], bench),
+        "config": config_block(bench.ws[0]),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "traffic_over_algorithmic": (traffic / (nbytes / args.steps)

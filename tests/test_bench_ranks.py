@@ -131,3 +131,17 @@ def test_traffic_record_needs_the_current_kernel_sources(tmp_path, monkeypatch):
     rec["kernel_sources"] = "0" * 16
     path.write_text(json.dumps(rec))
     assert bench.profiled_traffic("ragged_prefill_fp8")[0] is None
+
+
+def test_both_arms_name_the_same_config():
+    """The GPU arm's line and the reference arm's line carry the same config
+    block, derived from the workload alone."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    w = workloads.ragged_prefill_fp8()
+    c = bench.config_block(w)
+    assert c == bench.config_block(workloads.ragged_prefill_fp8())
+    assert c["replicas"] == len(bench.replica_workloads("ragged_prefill_fp8"))
+    assert c["workload"] == w.name and c["tokens_per_step"] == 9212 and "L2" in c["l2"]
