@@ -117,6 +117,10 @@ __device__ __forceinline__ void prefetch_task_lines(const WarpArgs& a, int w, co
 template <int POLICY, int STYLE, int NT, bool WV>
 __global__ void __launch_bounds__(NT, NT == kThreads ? 2 : 0) warp_append_kernel(const WarpArgs a) {
   constexpr int NW = NT / 32;  // warps per block
+  // a warp with one task waits on its own chain: the short form of the
+  // mean square (inv_rms_n) -- in the wide block, whose threads have no
+  // register cap (the short form needs more registers than 128)
+  constexpr int kForm = WV && NT == kWideThreads ? kSumShort : kSumMixed;
   extern __shared__ __align__(16) int smem[];
   float* s_w = reinterpret_cast<float*>(smem);  // 256 fp32 weights
   int* s_indptr = smem + 2 * kHeadDim;          // B + 1
@@ -291,11 +295,11 @@ __global__ void __launch_bounds__(NT, NT == kThreads ? 2 : 0) warp_append_kernel
             zero_tail_share(a.hp, r0.page, r0.slot_row, quad, a.qdiv, lane);
         }
         if (WV)
-          process_quad_cs<POLICY, STYLE>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, wq, l8,
-                                         gmask);
+          process_quad_cs<POLICY, STYLE, kForm>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, wq,
+                                                l8, gmask);
         else
-          process_quad_cs<POLICY, STYLE>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, s_w, l8,
-                                         gmask);
+          process_quad_cs<POLICY, STYLE, kForm>(a.hp, r0, 4 * quad, a.H, g, xa, xb, c0, s0, s_w,
+                                                l8, gmask);
         continue;
       }
       const int h = quad * 4 + g;
@@ -323,11 +327,11 @@ __global__ void __launch_bounds__(NT, NT == kThreads ? 2 : 0) warp_append_kernel
       // (a group past the last head only helps with the tail)
       const float* cs_row = a.cs + static_cast<int64_t>(r.pos) * a.hp.rot;
       if (WV)
-        process_quad<POLICY, STYLE, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, wg, l8,
-                                           gmask);
+        process_quad<POLICY, STYLE, false, kForm>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, wg,
+                                                  l8, gmask);
       else
-        process_quad<POLICY, STYLE, false>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row, s_w, l8,
-                                           gmask);
+        process_quad<POLICY, STYLE, false, kForm>(a.hp, r, 4 * quad, a.H, g, xa, xb, cs_row,
+                                                  s_w, l8, gmask);
     } else {
       // request task: the tail of a request without new rows (whose tail no
       // head task shares), or of every request when request tasks own tails

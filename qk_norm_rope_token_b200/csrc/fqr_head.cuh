@@ -368,7 +368,32 @@ __device__ __forceinline__ int quad_kind(const HeadParams& a, int h0) {
   return kAnyHead;
 }
 
-// 1 / sqrt(mean(x^2) + eps) of the head whose lane slices (8 float2 pairs,
+// The mean square of the head whose lane slices (8 float2 pairs) are y, over
+// the 8-lane group gmask: each value converted to binary64 by the hardware,
+// squared and summed there, then rounded once to fp32.  Valid for every input
+// (an Inf or a NaN propagates as in the definition); the slow path of
+// inv_rms_n.
+__device__ __forceinline__ float mean_square_general(const float2* y, unsigned gmask) {
+  double ss = 0.0;  // (one chain: a rare path, kept to few registers)
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const double u = y[j].x;
+    ss = fma(u, u, ss);
+    const double v = y[j].y;
+    ss = fma(v, v, ss);
+  }
+  ss += __shfl_xor_sync(gmask, ss, 4);
+  ss += __shfl_xor_sync(gmask, ss, 2);
+  ss += __shfl_xor_sync(gmask, ss, 1);
+  return __double2float_rn(ss * (1.0 / kHeadDim));
+}
+
+// How inv_rms_n forms the binary64 squares (both exact, see there):
+// kSumMixed takes fewer instructions (for throughput-bound kernels), kSumShort
+// has the shorter dependency chain (for a warp that holds a single task).
+enum SumForm { kSumMixed = 0, kSumShort = 1 };
+
+// 1 / sqrt(mean(x^2) + eps) of N heads whose lane slices (8 float2 pairs each,
 // BF16 values) are y, over the 8-lane group gmask.  The mean square is the
 // fp32 rounding of the exact mean of the squares: a BF16 value has 8
 // significant bits, its square 16, and the binary64 sum of a head's 128
@@ -377,18 +402,31 @@ __device__ __forceinline__ int quad_kind(const HeadParams& a, int h0) {
 // it.  One rounding to fp32, then +eps, the square root and the reciprocal,
 // each correctly rounded (rn_recip_sqrt).
 //
-// The squares are formed in binary64 from two conversions, to balance the
-// pipes: the first value of each pair by the hardware conversion, the second
-// by integer operations on its fp32 bits u -- for a BF16 value (8 significant
-// bits) the binary64 high word is ((u >> 3) & 0x0FFFFFFF) + ((1023 - 127) << 20)
-// with a zero low word (the sign is dropped: only the square is used).  That
-// is exact for every finite nonzero normal value; a zero or subnormal becomes
-// a value below 2^-126, whose square cannot reach the fp32 rounding of any
-// mean square that does not itself round to zero; an Inf becomes 2^128, as
-// good as infinite here (the mean square overflows, 1/sqrt gives 0); only a
-// NaN would turn finite, so when the mean square overflows, the head's values
-// are checked for a NaN (a rare branch), which then makes the result NaN.
-template <int N>
+// kSumMixed: the values go to binary64 by two conversions, to balance the
+// pipes -- the first value of each pair by the hardware conversion, the
+// second by integer operations on its fp32 bits u: for a BF16 value (8
+// significant bits) the binary64 high word is ((u >> 3) & 0x0FFFFFFF) +
+// ((1023 - 127) << 20) with a zero low word (the sign is dropped: only the
+// square is used).  That is exact for every finite nonzero normal value; a
+// zero or subnormal becomes a value below 2^-126, whose square cannot reach
+// the fp32 rounding of any mean square that does not itself round to zero;
+// an Inf becomes 2^128, as good as infinite here (the mean square overflows,
+// 1/sqrt gives 0); only a NaN would turn finite, so when the mean square
+// overflows, the head's values are checked for a NaN (a rare branch), which
+// then makes the result NaN.
+//
+// kSumShort: the squares are formed in fp32 (exact for |x| in [2^-63, 2^64):
+// 16 significant bits, no overflow or underflow) and moved to binary64 by a
+// shift: the binary32 pattern of a non-negative p shifted right by 3 is the
+// high word of the binary64 value p * 2^-896 with a zero low word -- exact for
+// every finite p, zero and subnormal included (the exponent fields line up,
+// without the bias difference).  The sum is scaled back by 2^889 (2^896 over
+// the 128 values), exactly.  A mean square outside [2^-60, 2^121) (which any
+// |x| >= 2^64, an Inf or a NaN puts above, and only heads of tiny values
+// below) is recomputed by mean_square_general on a rare branch: inside that
+// range every value below 2^-63 is too small to reach the fp32 rounding of
+// the exact mean wherever the span condition above holds.
+template <int N, int FORM = kSumMixed>
 __device__ __forceinline__ void inv_rms_n(float2 (*y)[8], float eps, unsigned gmask, float* inv) {
   double ss[N];
 #pragma unroll
@@ -396,12 +434,22 @@ __device__ __forceinline__ void inv_rms_n(float2 (*y)[8], float eps, unsigned gm
     double s[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const uint32_t uy = __float_as_uint(y[n][j].y);
-      const double u = y[n][j].x;
-      const double v =
-          __hiloint2double(static_cast<int>(__umulhi(uy & 0x7FFF0000u, 1u << 29) + 0x38000000u), 0);
-      s[(j & 1) * 2] = fma(u, u, s[(j & 1) * 2]);
-      s[(j & 1) * 2 + 1] = fma(v, v, s[(j & 1) * 2 + 1]);
+      double u, v;
+      if (FORM == kSumMixed) {
+        u = y[n][j].x;
+        v = __hiloint2double(
+            static_cast<int>(__umulhi(__float_as_uint(y[n][j].y) & 0x7FFF0000u, 1u << 29) +
+                             0x38000000u),
+            0);
+        s[(j & 1) * 2] = fma(u, u, s[(j & 1) * 2]);
+        s[(j & 1) * 2 + 1] = fma(v, v, s[(j & 1) * 2 + 1]);
+      } else {
+        const float2 p = mul2(y[n][j], y[n][j]);
+        u = __hiloint2double(static_cast<int>(__float_as_uint(p.x) >> 3), 0);
+        v = __hiloint2double(static_cast<int>(__float_as_uint(p.y) >> 3), 0);
+        s[(j & 1) * 2] += u;
+        s[(j & 1) * 2 + 1] += v;
+      }
     }
     ss[n] = (s[0] + s[1]) + (s[2] + s[3]);
   }
@@ -412,12 +460,21 @@ __device__ __forceinline__ void inv_rms_n(float2 (*y)[8], float eps, unsigned gm
   }
 #pragma unroll
   for (int n = 0; n < N; ++n) {
-    float ms = __double2float_rn(ss[n] * (1.0 / kHeadDim));
-    if (__builtin_expect(ms == INFINITY, 0)) {  // the whole 8-lane group agrees on ms
-      bool nan = false;
+    float ms;
+    if (FORM == kSumMixed) {
+      ms = __double2float_rn(ss[n] * (1.0 / kHeadDim));
+      if (__builtin_expect(ms == INFINITY, 0)) {  // the whole 8-lane group agrees on ms
+        bool nan = false;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) nan |= isnan(y[n][j].x) || isnan(y[n][j].y);
-      if (__any_sync(gmask, nan)) ms = __int_as_float(0x7FC00000);
+        for (int j = 0; j < 8; ++j) nan |= isnan(y[n][j].x) || isnan(y[n][j].y);
+        if (__any_sync(gmask, nan)) ms = __int_as_float(0x7FC00000);
+      }
+    } else {
+      ms = __double2float_rn(ss[n] * 0x1p889);
+      // ms in [2^-60, 2^121) as one unsigned compare of the bit patterns; the
+      // whole 8-lane group agrees on ms
+      if (__builtin_expect(__float_as_uint(ms) - 0x21800000u >= 0x7C000000u - 0x21800000u, 0))
+        ms = mean_square_general(y[n], gmask);
     }
     inv[n] = rn_recip_sqrt(__fadd_rn(ms, eps));
   }
@@ -491,13 +548,13 @@ __device__ __forceinline__ void output_qk_head(const HeadParams& a, const RowCtx
 // kKHead) of row r at once, from their lane slices y (unpacked): the heads'
 // dependency chains interleave, and they share the cos/sin values and the
 // norm weights.
-template <int POLICY, int STYLE, int KIND, int N, class W>
+template <int POLICY, int STYLE, int KIND, int N, int FORM, class W>
 __device__ __forceinline__ void process_qk_heads(const HeadParams& a, const RowCtx& r, const int* h,
                                                  float2 (*y)[8], const float2* c, const float2* s,
                                                  const W& wts, int l8, unsigned gmask) {
   if (KIND == kQHead ? a.has_qw : a.has_kw) {
     float inv[N];
-    inv_rms_n<N>(y, a.eps, gmask, inv);
+    inv_rms_n<N, FORM>(y, a.eps, gmask, inv);
     float2 w[8];
     load_weights(wts, KIND == kQHead, l8, w);
 #pragma unroll
@@ -519,7 +576,7 @@ __device__ __forceinline__ void process_qk_heads(const HeadParams& a, const RowC
 // the 8-lane group.  KIND: the head's kind when the caller knows it
 // (HeadKind).  Request tails are zeroed by the callers (zero_tail_share), not
 // here.
-template <int POLICY, int STYLE, int KIND = kAnyHead, class W>
+template <int POLICY, int STYLE, int KIND = kAnyHead, int FORM = kSumMixed, class W>
 __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCtx& r, int h,
                                                 uint4 xa, uint4 xb, const float2* c,
                                                 const float2* s, const W& wts, int l8,
@@ -551,27 +608,28 @@ __device__ __forceinline__ void process_head_cs(const HeadParams& a, const RowCt
     for (int j = 0; j < 8; ++j) yy[0][j] = y[j];
     const bool is_q = KIND == kQHead || (KIND == kAnyHead && h < a.Hq);
     if (is_q)
-      process_qk_heads<POLICY, STYLE, kQHead, 1>(a, r, &h, yy, c, s, wts, l8, gmask);
+      process_qk_heads<POLICY, STYLE, kQHead, 1, FORM>(a, r, &h, yy, c, s, wts, l8, gmask);
     else
-      process_qk_heads<POLICY, STYLE, kKHead, 1>(a, r, &h, yy, c, s, wts, l8, gmask);
+      process_qk_heads<POLICY, STYLE, kKHead, 1, FORM>(a, r, &h, yy, c, s, wts, l8, gmask);
   }
 }
 
 // As process_head_cs, loading the cos/sin values from cs_row first (V heads
 // need none).
-template <int POLICY, int STYLE, bool CS_SMEM, int KIND = kAnyHead, class W>
+template <int POLICY, int STYLE, bool CS_SMEM, int KIND = kAnyHead, int FORM = kSumMixed,
+          class W>
 __device__ __forceinline__ void process_head(const HeadParams& a, const RowCtx& r, int h,
                                              uint4 xa, uint4 xb, const float* cs_row,
                                              const W& wts, int l8, unsigned gmask) {
   float2 c[4], s[4];
   if (KIND == kQHead || KIND == kKHead || (KIND == kAnyHead && h < a.Hq + a.Hkv))
     load_cs<STYLE, CS_SMEM>(cs_row, a.rot, l8, c, s);
-  process_head_cs<POLICY, STYLE, KIND>(a, r, h, xa, xb, c, s, wts, l8, gmask);
+  process_head_cs<POLICY, STYLE, KIND, FORM>(a, r, h, xa, xb, c, s, wts, l8, gmask);
 }
 
 // process_head_cs for one quad whose first head is h0 (warp-uniform), with
 // the cos/sin values already loaded; see process_quad.
-template <int POLICY, int STYLE, class W>
+template <int POLICY, int STYLE, int FORM = kSumMixed, class W>
 __device__ __forceinline__ void process_quad_cs(const HeadParams& a, const RowCtx& r, int h0,
                                                 int nheads, int g, uint4 xa, uint4 xb,
                                                 const float2* c, const float2* s, const W& wts,
@@ -579,19 +637,19 @@ __device__ __forceinline__ void process_quad_cs(const HeadParams& a, const RowCt
   const int h = h0 + g;
   const int kind = h0 + 4 <= nheads ? quad_kind(a, h0) : kAnyHead;
   if (kind == kQHead)
-    process_head_cs<POLICY, STYLE, kQHead>(a, r, h, xa, xb, c, s, wts, l8, gmask);
+    process_head_cs<POLICY, STYLE, kQHead, FORM>(a, r, h, xa, xb, c, s, wts, l8, gmask);
   else if (kind == kKHead)
-    process_head_cs<POLICY, STYLE, kKHead>(a, r, h, xa, xb, c, s, wts, l8, gmask);
+    process_head_cs<POLICY, STYLE, kKHead, FORM>(a, r, h, xa, xb, c, s, wts, l8, gmask);
   else if (kind == kVHead)
-    process_head_cs<POLICY, STYLE, kVHead>(a, r, h, xa, xb, c, s, wts, l8, gmask);
+    process_head_cs<POLICY, STYLE, kVHead, FORM>(a, r, h, xa, xb, c, s, wts, l8, gmask);
   else if (h < nheads)
-    process_head_cs<POLICY, STYLE, kAnyHead>(a, r, h, xa, xb, c, s, wts, l8, gmask);
+    process_head_cs<POLICY, STYLE, kAnyHead, FORM>(a, r, h, xa, xb, c, s, wts, l8, gmask);
 }
 
 // process_head for one quad whose first head is h0 (warp-uniform): the kind
 // is decided once for the warp when all four heads exist; otherwise each
 // group decides for its own head (h0 + g < nheads).
-template <int POLICY, int STYLE, bool CS_SMEM, class W>
+template <int POLICY, int STYLE, bool CS_SMEM, int FORM = kSumMixed, class W>
 __device__ __forceinline__ void process_quad(const HeadParams& a, const RowCtx& r, int h0,
                                              int nheads, int g, uint4 xa, uint4 xb,
                                              const float* cs_row, const W& wts, int l8,
@@ -599,13 +657,13 @@ __device__ __forceinline__ void process_quad(const HeadParams& a, const RowCtx& 
   const int h = h0 + g;
   const int kind = h0 + 4 <= nheads ? quad_kind(a, h0) : kAnyHead;
   if (kind == kQHead)
-    process_head<POLICY, STYLE, CS_SMEM, kQHead>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kQHead, FORM>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
   else if (kind == kKHead)
-    process_head<POLICY, STYLE, CS_SMEM, kKHead>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kKHead, FORM>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
   else if (kind == kVHead)
-    process_head<POLICY, STYLE, CS_SMEM, kVHead>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kVHead, FORM>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
   else if (h < nheads)
-    process_head<POLICY, STYLE, CS_SMEM, kAnyHead>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
+    process_head<POLICY, STYLE, CS_SMEM, kAnyHead, FORM>(a, r, h, xa, xb, cs_row, wts, l8, gmask);
 }
 
 // Zero the whole tail (rows [last+1, P), all heads) of request b's last page in

@@ -336,6 +336,13 @@ def _special_heads(w, seed):
         lambda x, g: (x.__setitem__(slice(None), 0), x.__setitem__(77, 0x3F80)),          # one-hot
         lambda x, g: x.__setitem__(slice(None), np.where(g.random(D) < 0.5, 0x7149, 0x0DA2)),  # 1e30 / 1e-30
         lambda x, g: x.__setitem__(slice(None), x & 0x80FF | 0x0080),  # tiny normals
+        # the bounds of the fp32-squares form's range: squares near 2^-60
+        lambda x, g: x.__setitem__(slice(None), x & 0x807F | 0x3080),
+        # values whose fp32 squares round (below 2^-63) beside N(0, 1) values
+        lambda x, g: x.__setitem__(slice(None), np.where(g.random(D) < 0.5, x, 0x1CC1)),
+        # one square just below the fp32 overflow, then one far above it
+        lambda x, g: x.__setitem__(40, 0x5F35),
+        lambda x, g: (x.__setitem__(40, 0x5F35), x.__setitem__(41, 0x6780)),
     ]
     heads = list(range(w.Hq)) + list(range(w.Hq, w.Hq + w.Hkv))
     r = 0
@@ -360,4 +367,17 @@ def test_special_values_in_normed_heads(policy, schedule):
                               cos_sin_rows=128, k_scale=0.05, v_scale=0.05)
     _special_heads(w, 5)
     _, rep = run_and_check(w, schedule=schedule)
+    assert not rep.get("flagged")
+
+
+@pytest.mark.parametrize("policy", [0, 1])
+def test_special_values_in_wide_block_heads(policy):
+    """The same special values in a decode batch that takes the latency
+    schedule's wide block, whose warps (one task each) form the mean square
+    from fp32 squares: its rare-branch fallback against the oracle."""
+    w = _wide_block_decode(policy, 0)
+    _special_heads(w, 6)
+    plan = AppendRun(w, schedule=0).plan()
+    assert plan["block_threads"] == 384 and plan["warp_check"] == 1
+    _, rep = run_and_check(w, schedule=1)
     assert not rep.get("flagged")
