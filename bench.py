@@ -491,7 +491,7 @@ def e2e_measure(torch, fqr, bench, steps):
     out_shapes = {"out_q": (tuple(bench.reps[0]["out_q"].shape), bench.reps[0]["out_q"].dtype),
                   "flags": ((w0.B,), torch.int32)}
     if w0.quant_policy == 1:
-        out_shapes["q_scale"] = ((w0.T, w0.Hq), torch.float32)
+        out_shapes["q_scale"] = (tuple(w0.q_scale_shape), torch.float32)
     kw = bench.kw_for(w0, {"q_scale": None})
     kw.pop("q_scale", None)
     sa = fqr.StagedAppend(in_shapes, out_shapes, dev, depth=3, cos_sin_cache=bench.cs,
@@ -524,18 +524,22 @@ def e2e_measure(torch, fqr, bench, steps):
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
     assert int(host_out[(steps - 1) % R]["flags"].abs().max()) == 0
+    # the host outputs of the first replica's last step, for the check in the
+    # cpu_baseline leg (outside the timed region)
+    sample = {k: v.clone() for k, v in host_out[0].items() if not k.startswith("_")}
     sa.close()
     return {"value": bench.T * steps / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps,
             "api": "qk_norm_rope_token_b200.StagedAppend over the library's native pipeline "
-                   "(fqr_pipeline_*: 3 streams, 3 staging slots, one copy each way per step)"}
+                   "(fqr_pipeline_*: 3 streams, 3 staging slots, one copy each way per step)"}, sample
 
 
 # ----------------------------------------------------------- CPU baselines
 
-def oracle_sample(w, budget_s, max_calls=None):
+def oracle_sample(w, budget_s, max_calls=None, outputs=None):
     """Time the oracle as it stands on whole calls of workload w (host caches
-    allocated lazily: only the pages a call touches are materialised)."""
+    allocated lazily: only the pages a call touches are materialised).
+    outputs: a dict that receives the last call's out_q, q_scale and flags."""
     import oracle
     es = w.kv_esize
     dt = np.uint16 if es == 2 else np.uint8
@@ -551,14 +555,29 @@ def oracle_sample(w, budget_s, max_calls=None):
         el = time.perf_counter() - t0
         if (max_calls and calls >= max_calls) or (not max_calls and el >= budget_s):
             break
+    if outputs is not None:
+        outputs.update(out_q=oq, q_scale=qs, flags=fl)
     return calls, el
 
 
-def cpu_baseline(w, budget_s):
-    calls, el = oracle_sample(w, budget_s)
-    return {"value": w.T * calls / el, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{calls} whole calls of {w.name} ({w.T} tokens each), "
-                      f"{el:.1f} s single-threaded C oracle (fp32, -O2, no FMA)"}
+def cpu_baseline(w, budget_s, e2e_sample=None):
+    """The oracle on whole calls of w for about budget_s; with e2e_sample (the
+    e2e leg's host outputs of one step on w), also whether they are
+    bit-identical to the oracle's."""
+    outs = {}
+    calls, el = oracle_sample(w, budget_s, outputs=outs)
+    res = {"value": w.T * calls / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"{calls} whole calls of {w.name} ({w.T} tokens each), "
+                     f"{el:.1f} s single-threaded C oracle (fp32, -O2, no FMA)"}
+    if e2e_sample is not None:
+        same = {}
+        for k in ("out_q", "q_scale", "flags"):
+            if k in e2e_sample:
+                got = e2e_sample[k].numpy()
+                same[k] = bool(got.shape == outs[k].shape
+                               and got.tobytes() == np.ascontiguousarray(outs[k]).tobytes())
+        res["e2e_check"] = {"against": "the oracle's outputs of the same call", "identical": same}
+    return res
 
 
 def _oracle_worker(job):
@@ -745,7 +764,7 @@ def main(argv=None):
     achieved = nbytes / args.steps / per_launch_s / 1e9
     traffic, traffic_parts = profiled_traffic(args.workload)
 
-    e2e = e2e_measure(torch, fqr, bench, min(args.e2e_steps, max(args.steps, 1)))
+    e2e, e2e_sample = e2e_measure(torch, fqr, bench, min(args.e2e_steps, max(args.steps, 1)))
     e2e_ms = max_over_ranks(torch, dist, e2e["ms_per_step"], dev)
     e2e["value"] = world * bench.T / (e2e_ms / 1e3)
     per_config = None
@@ -753,7 +772,8 @@ def main(argv=None):
         per_config = measure_per_config(torch, fqr, dev, peak)
     cpu = cpu_all = None
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        cpu = cpu_baseline(bench.ws[0], args.cpu_seconds)
+        cpu = cpu_baseline(bench.ws[0], args.cpu_seconds, e2e_sample)
+        e2e["check"] = cpu.pop("e2e_check")
         cpu_all = cpu_baseline_all_cores(bench.ws[0], args.cpu_seconds)
     if dist is not None:
         barrier()
