@@ -37,6 +37,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -122,12 +123,21 @@ APPEND_KERNEL_SOURCES = ("fqr_append.cu", "fqr_append_pipe.cu", "fqr_append_warp
                          "fqr_device.cuh", "fqr_head.cuh", "fqr_launch.h")
 
 
+def _code_tokens(text: str) -> str:
+    """A source file without its comments and with whitespace collapsed (the
+    sources hold no string literal with a comment marker)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(names=APPEND_KERNEL_SOURCES) -> str:
+    """Hash of the append kernels' code: comments and layout do not change it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "qk_norm_rope_token_b200", "csrc")
     for name in sorted(names):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update((name + "\n" + _code_tokens(f.read())).encode())
     return h.hexdigest()[:16]
 
 

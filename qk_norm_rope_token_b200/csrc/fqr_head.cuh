@@ -418,10 +418,11 @@ enum SumForm { kSumMixed = 0, kSumShort = 1 };
 // kSumShort: the squares are formed in fp32 (exact for |x| in [2^-63, 2^64):
 // 16 significant bits, no overflow or underflow) and moved to binary64 by a
 // shift: the binary32 pattern of a non-negative p shifted right by 3 is the
-// high word of the binary64 value p * 2^-896 with a zero low word -- exact for
-// every finite p, zero and subnormal included (the exponent fields line up,
-// without the bias difference).  The sum is scaled back by 2^889 (2^896 over
-// the 128 values), exactly.  A mean square outside [2^-60, 2^121) (which any
+// high word of the binary64 value p * 2^-896 (the exponent fields line up,
+// without the bias difference; zero and subnormal patterns too) with a low
+// word of p's three lowest bits -- zero for such an exact square, so the low
+// word is left zero (a smaller, rounded square loses bits below 2^-146).  The
+// sum is scaled back by 2^889 (2^896 over the 128 values), exactly.  A mean square outside [2^-60, 2^121) (which any
 // |x| >= 2^64, an Inf or a NaN puts above, and only heads of tiny values
 // below) is recomputed by mean_square_general on a rare branch: inside that
 // range every value below 2^-63 is too small to reach the fp32 rounding of

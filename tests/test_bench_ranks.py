@@ -145,3 +145,15 @@ def test_both_arms_name_the_same_config():
     assert c == bench.config_block(workloads.ragged_prefill_fp8())
     assert c["replicas"] == len(bench.replica_workloads("ragged_prefill_fp8"))
     assert c["workload"] == w.name and c["tokens_per_step"] == 9212 and "L2" in c["l2"]
+
+
+def test_kernel_source_hash_ignores_comments_and_layout():
+    """The hash that keys the traffic record follows the kernels' code only."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    a = "int f(int x) {  // the identity\n  return x; /* no\n change */ }\n"
+    b = "int f(int x) {\n/* a different\n comment */ return x;\n}"
+    assert bench._code_tokens(a) == bench._code_tokens(b) == "int f(int x) { return x; }"
+    assert bench._code_tokens("return x + 1;") != bench._code_tokens("return x;")
+    assert bench.kernel_source_hash() == bench.kernel_source_hash()
