@@ -157,3 +157,29 @@ def test_kernel_source_hash_ignores_comments_and_layout():
     assert bench._code_tokens(a) == bench._code_tokens(b) == "int f(int x) { return x; }"
     assert bench._code_tokens("return x + 1;") != bench._code_tokens("return x;")
     assert bench.kernel_source_hash() == bench.kernel_source_hash()
+
+
+def test_cpu_leg_checks_the_e2e_outputs_byte_for_byte():
+    """The cpu_baseline leg compares the e2e leg's host outputs of one step
+    with the oracle's outputs of the same call: identical when they are the
+    oracle's own, not identical once one byte of out_q differs."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import numpy as np
+    import oracle
+    import workloads
+    w = workloads.APPEND_CONFIGS["tiny_decode_bf16"]()
+    es = w.kv_esize
+    dt = np.uint16 if es == 2 else np.uint8
+    kc = np.zeros((w.num_pages, w.page_size, w.Hkv, 128), dt)
+    vc = np.zeros_like(kc)
+    oq, qs, fl = oracle.new_outputs(w)
+    assert oracle.append_paged(w, kc, vc, oq, None, fl) == 0
+    sample = {"out_q": torch.from_numpy(oq.view(np.int16).copy()),
+              "flags": torch.from_numpy(fl.copy())}
+    res = bench.cpu_baseline(w, 0.05, sample)
+    assert res["e2e_check"]["identical"] == {"out_q": True, "flags": True}
+    sample["out_q"].view(-1)[7] ^= 1
+    res = bench.cpu_baseline(w, 0.05, sample)
+    assert res["e2e_check"]["identical"] == {"out_q": False, "flags": True}
